@@ -1,0 +1,204 @@
+// Host side of the librola C ABI: status strings, shape validation, the
+// kept-block rule, rotary frequency table, driver entry point for tensor-map
+// encoding, and the whole-layer entry points that chain the kernels.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "rola_common.cuh"
+#include "rola_internal.h"
+
+namespace rola_internal {
+
+rola_status_t check_shape(const rola_shape_t* s) {
+  if (!s) return ROLA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->T < 1 || s->Hg < 1 || s->W < 1 || s->d < 1 || s->r < 1 ||
+      s->block < 1)
+    return ROLA_ERR_INVALID_ARG;
+  const long long N = (long long)s->T * s->Hg * s->W;
+  if (N != s->N || N > (1LL << 30)) return ROLA_ERR_INVALID_ARG;
+  if ((long long)s->B * N * s->H * s->d >= (1LL << 40)) return ROLA_ERR_INVALID_ARG;
+  const int nb = (int)((N + s->block - 1) / s->block);
+  if (s->k_b < 1 || s->k_b > nb) return ROLA_ERR_INVALID_ARG;
+  if (s->r % 2 != 0 || s->r > s->d) return ROLA_ERR_INVALID_ARG;
+  if (!(s->rope_base > 0.f) || !isfinite(s->rope_base)) return ROLA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return ROLA_ERR_UNSUPPORTED;
+  if (s->block != 64 && s->block != 128) return ROLA_ERR_UNSUPPORTED;
+  if (s->r != 16 && s->r != 32) return ROLA_ERR_UNSUPPORTED;
+  return ROLA_OK;
+}
+
+LayerWs layer_ws(const rola_shape_t* s) {
+  LayerWs w{};
+  const size_t nb = (size_t)rola_num_blocks(s);
+  const size_t BH = (size_t)s->B * s->H;
+  size_t off = 0;
+  w.select = off;
+  off += round_up(rola_select_workspace_bytes(s), 256);
+  w.idx = off;
+  off += round_up(BH * nb * s->k_b * sizeof(int32_t), 256);
+  w.S_blk = off;
+  off += round_up(BH * nb * s->r * s->d * sizeof(float), 256);
+  w.z_blk = off;
+  off += round_up(BH * nb * s->r * sizeof(float), 256);
+  w.S_glb = off;
+  off += round_up(BH * s->r * s->d * sizeof(float), 256);
+  w.z_glb = off;
+  off += round_up(BH * s->r * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+}  // namespace rola_internal
+
+namespace rola_host {
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int rope_frequencies(int r, float base, double* freq, int* axis) {
+  const int rh = 2 * (r / 6);
+  const int split[3] = {r - 2 * rh, rh, rh};
+  int p = 0;
+  for (int ax = 0; ax < 3; ++ax)
+    for (int m = 0; m < split[ax] / 2; ++m) {
+      freq[p] = pow((double)base, -2.0 * m / split[ax]);
+      axis[p] = ax;
+      ++p;
+    }
+  return p;
+}
+
+}  // namespace rola_host
+
+using rola_internal::check_shape;
+
+extern "C" const char* rola_status_string(rola_status_t s) {
+  switch (s) {
+    case ROLA_OK: return "ok";
+    case ROLA_ERR_INVALID_ARG: return "invalid argument";
+    case ROLA_ERR_UNSUPPORTED: return "unsupported shape";
+    case ROLA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case ROLA_ERR_CUDA: return "CUDA error";
+    case ROLA_ERR_ALIGNMENT: return "pointer misaligned";
+  }
+  return "unknown status";
+}
+
+extern "C" int32_t rola_num_blocks(const rola_shape_t* s) {
+  if (!s || s->block < 1 || s->N < 1) return -1;
+  return (int32_t)(((long long)s->N + s->block - 1) / s->block);
+}
+
+extern "C" int32_t rola_kb_from_sparsity(int32_t n_blocks, int32_t sparsity_permille) {
+  if (n_blocks < 1 || sparsity_permille < 0 || sparsity_permille >= 1000) return -1;
+  const long long keep = (long long)(1000 - sparsity_permille) * n_blocks;
+  return (int32_t)((keep + 999) / 1000);
+}
+
+extern "C" size_t rola_layer_workspace_bytes(const rola_shape_t* s) {
+  if (check_shape(s) != ROLA_OK) return 0;
+  return rola_internal::layer_ws(s).total;
+}
+
+extern "C" rola_status_t rola_layer_fwd(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
+                                        const uint16_t* v, const uint16_t* P, const float* gate,
+                                        uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                                        int32_t* dev_err, void* stream) {
+  rola_status_t st = check_shape(s);
+  if (st != ROLA_OK) return st;
+  const rola_internal::LayerWs L = rola_internal::layer_ws(s);
+  if (!ws || ws_bytes < L.total || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
+  char* base = reinterpret_cast<char*>(ws);
+  int32_t* idx = reinterpret_cast<int32_t*>(base + L.idx);
+  float* S_blk = reinterpret_cast<float*>(base + L.S_blk);
+  float* z_blk = reinterpret_cast<float*>(base + L.z_blk);
+  float* S_glb = reinterpret_cast<float*>(base + L.S_glb);
+  float* z_glb = reinterpret_cast<float*>(base + L.z_glb);
+  st = rola_select_blocks(s, q, k, idx, nullptr, base + L.select, L.idx - L.select, stream);
+  if (st != ROLA_OK) return st;
+  st = rola_block_states(s, k, v, P, S_blk, z_blk, S_glb, z_glb, stream);
+  if (st != ROLA_OK) return st;
+  st = rola_attention_fwd(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
+                          stream);
+  if (st != ROLA_OK) return st;
+  if (idx_out) {
+    const size_t bytes = (size_t)s->B * s->H * rola_num_blocks(s) * s->k_b * sizeof(int32_t);
+    if (cudaMemcpyAsync(idx_out, idx, bytes, cudaMemcpyDeviceToDevice,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return ROLA_ERR_CUDA;
+  }
+  return ROLA_OK;
+}
+
+namespace {
+struct HostWs {
+  size_t q, k, v, P, gate, out, layer, total;
+};
+HostWs host_ws(const rola_shape_t* s) {
+  using rola_internal::round_up;
+  HostWs w{};
+  const size_t act = (size_t)s->B * s->N * s->H * s->d * sizeof(uint16_t);
+  size_t off = 0;
+  w.q = off; off += round_up(act, 256);
+  w.k = off; off += round_up(act, 256);
+  w.v = off; off += round_up(act, 256);
+  w.out = off; off += round_up(act, 256);
+  w.P = off; off += round_up((size_t)s->H * s->d * s->r * sizeof(uint16_t), 256);
+  w.gate = off; off += round_up((size_t)s->H * sizeof(float), 256);
+  w.layer = off; off += rola_internal::layer_ws(s).total;
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+extern "C" size_t rola_layer_host_workspace_bytes(const rola_shape_t* s) {
+  if (check_shape(s) != ROLA_OK) return 0;
+  return host_ws(s).total;
+}
+
+extern "C" rola_status_t rola_layer_fwd_host(const rola_shape_t* s, const uint16_t* q_host,
+                                             const uint16_t* k_host, const uint16_t* v_host,
+                                             const uint16_t* P_host, const float* gate_host,
+                                             uint16_t* out_host, void* ws, size_t ws_bytes,
+                                             int32_t* dev_err, void* stream) {
+  rola_status_t st = check_shape(s);
+  if (st != ROLA_OK) return st;
+  if (!q_host || !k_host || !v_host || !P_host || !gate_host || !out_host)
+    return ROLA_ERR_INVALID_ARG;
+  const HostWs w = host_ws(s);
+  if (!ws || ws_bytes < w.total || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  char* base = reinterpret_cast<char*>(ws);
+  const size_t act = (size_t)s->B * s->N * s->H * s->d * sizeof(uint16_t);
+  const size_t pbytes = (size_t)s->H * s->d * s->r * sizeof(uint16_t);
+  if (cudaMemcpyAsync(base + w.q, q_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(base + w.k, k_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(base + w.v, v_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(base + w.P, P_host, pbytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(base + w.gate, gate_host, (size_t)s->H * sizeof(float),
+                      cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  st = rola_layer_fwd(s, reinterpret_cast<uint16_t*>(base + w.q),
+                      reinterpret_cast<uint16_t*>(base + w.k),
+                      reinterpret_cast<uint16_t*>(base + w.v),
+                      reinterpret_cast<uint16_t*>(base + w.P), reinterpret_cast<float*>(base + w.gate),
+                      reinterpret_cast<uint16_t*>(base + w.out), nullptr, base + w.layer,
+                      w.total - w.layer, dev_err, stream);
+  if (st != ROLA_OK) return st;
+  if (cudaMemcpyAsync(out_host, base + w.out, act, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  return ROLA_OK;
+}

@@ -1,0 +1,237 @@
+// Block selector: mean-pool q and k per block (float64, exact block sums of
+// bf16), score every query block against every key block with the float64
+// tensor-core path (DMMA m8n8k4), and keep the top k_b key blocks per query
+// block by (-score, index), emitted ascending.
+//
+// SparkDiffusion write-up (0539edu.com news page), section 01: sparse
+// attention keeps only the important query-key blocks; section 05: RoLA's
+// sparse branch keeps the high-energy query-key block interactions.  The
+// mean-pooled score is this library's concrete selector (the pages give none).
+#include <float.h>
+#include <math.h>
+
+#include "rola_common.cuh"
+#include "rola_internal.h"
+
+namespace rola {
+
+// ---------------------------------------------------------------- pooling
+// grid (n_blocks, B, 2 [q or k]), 256 threads; each thread owns 8 adjacent
+// bf16 columns of the [N, H*d] token rows and sums the block's valid tokens.
+__global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ q,
+                                                   const uint16_t* __restrict__ k,
+                                                   double* __restrict__ qbar,
+                                                   double* __restrict__ kbar, int N, int H, int d,
+                                                   int bs, int nb) {
+  const int blk = blockIdx.x, b = blockIdx.y;
+  const uint16_t* src = blockIdx.z == 0 ? q : k;
+  double* dst = blockIdx.z == 0 ? qbar : kbar;
+  const int HD = H * d;
+  const int n0 = blk * bs, n1 = min(N, n0 + bs);
+  const double cnt = (double)(n1 - n0);
+  const size_t row_stride = (size_t)HD / 8;  // in uint4
+  for (int c8 = threadIdx.x; c8 < HD / 8; c8 += blockDim.x) {
+    double acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+    const uint4* p = reinterpret_cast<const uint4*>(src + ((size_t)b * N + n0) * HD) + c8;
+    int n = n0;
+    for (; n + 8 <= n1; n += 8) {
+      uint4 u[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) u[t] = __ldg(p + (size_t)t * row_stride);
+      p += 8 * row_stride;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const uint32_t w[4] = {u[t].x, u[t].y, u[t].z, u[t].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += (double)bf16_lo(w[i]);
+          acc[2 * i + 1] += (double)bf16_hi(w[i]);
+        }
+      }
+    }
+    for (; n < n1; ++n) {
+      const uint4 u = __ldg(p);
+      p += row_stride;
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += (double)bf16_lo(w[i]);
+        acc[2 * i + 1] += (double)bf16_hi(w[i]);
+      }
+    }
+    const int col = c8 * 8, h = col / d, c = col % d;
+    double* o = dst + (((size_t)b * H + h) * nb + blk) * d + c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = acc[i] / cnt;
+  }
+}
+
+// ---------------------------------------------------------------- scores
+// sigma[b,h,a,j] = qbar[b,h,a,:] . kbar[b,h,j,:] / sqrt(d) in float64.
+// CTA tile 64 x 64 (4 warps of 32 x 32), d staged through shared memory in
+// chunks of 32; each warp runs 4 x 4 DMMA m8n8k4 tiles per k-step of 4.
+constexpr int kScTile = 64, kScChunk = 32, kScStride = 36;  // stride keeps DMMA loads conflict-free
+
+ROLA_DEV void dmma_8x8x4(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar,
+                                                    const double* __restrict__ kbar,
+                                                    double* __restrict__ sigma, int H, int d,
+                                                    int nb) {
+  __shared__ double sA[kScTile * kScStride];
+  __shared__ double sB[kScTile * kScStride];
+  const int bh = blockIdx.z;
+  const int row0 = blockIdx.y * kScTile, col0 = blockIdx.x * kScTile;
+  const double* A = qbar + (size_t)bh * nb * d;
+  const double* Bm = kbar + (size_t)bh * nb * d;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+  double acc[4][4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+
+  for (int c0 = 0; c0 < d; c0 += kScChunk) {
+    for (int e = threadIdx.x; e < kScTile * kScChunk; e += blockDim.x) {
+      const int r = e / kScChunk, c = e % kScChunk;
+      sA[r * kScStride + c] = (row0 + r < nb) ? A[(size_t)(row0 + r) * d + c0 + c] : 0.0;
+      sB[r * kScStride + c] = (col0 + r < nb) ? Bm[(size_t)(col0 + r) * d + c0 + c] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kScChunk; kk += 4) {
+      double af[4], bf[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        af[i] = sA[(wr + 8 * i + (lane >> 2)) * kScStride + kk + (lane & 3)];
+        bf[i] = sB[(wc + 8 * i + (lane >> 2)) * kScStride + kk + (lane & 3)];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j], af[i], bf[j]);
+    }
+    __syncthreads();
+  }
+  const double rs = sqrt((double)d);
+  double* S = sigma + (size_t)bh * nb * nb;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = row0 + wr + 8 * i + (lane >> 2);
+      const int c = col0 + wc + 8 * j + 2 * (lane & 3);
+      if (r < nb) {
+        if (c < nb) S[(size_t)r * nb + c] = acc[i][j][0] / rs;
+        if (c + 1 < nb) S[(size_t)r * nb + c + 1] = acc[i][j][1] / rs;
+      }
+    }
+}
+
+// ---------------------------------------------------------------- top-k
+// One warp per (b, h, query block).  Lane l holds scores of blocks l, l+32, ...
+// (n_blocks <= 32 * 32).  k_b rounds of a warp arg-max by (score desc, index
+// asc); the chosen set is then written in ascending block order.
+constexpr int kMaxPerLane = 32;
+
+__global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ sigma,
+                                                   int32_t* __restrict__ idx, int rows, int nb,
+                                                   int kb) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const double* s = sigma + (size_t)warp * nb;
+  int32_t* out = idx + (size_t)warp * kb;
+  const int nper = (nb + 31) / 32;
+  double v[kMaxPerLane];
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int j = i * 32 + lane;
+    v[i] = (i < nper && j < nb) ? s[j] : -DBL_MAX;
+  }
+  uint32_t taken = 0;
+  if (kb >= nb) {
+    taken = 0xffffffffu;
+  } else {
+    for (int round = 0; round < kb; ++round) {
+      double best = -INFINITY;
+      int bidx = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i) {
+        const int j = i * 32 + lane;
+        if (i < nper && j < nb && !((taken >> i) & 1u) && (v[i] > best || bidx == 0x7fffffff)) {
+          if (bidx == 0x7fffffff || v[i] > best) {
+            best = v[i];
+            bidx = j;
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
+        if (oi != 0x7fffffff && (bidx == 0x7fffffff || ob > best || (ob == best && oi < bidx))) {
+          best = ob;
+          bidx = oi;
+        }
+      }
+      if (bidx != 0x7fffffff && (bidx & 31) == lane) taken |= 1u << (bidx >> 5);
+    }
+  }
+  int pos = 0;
+  for (int i = 0; i < nper; ++i) {
+    const int j = i * 32 + lane;
+    const bool mine = j < nb && ((taken >> i) & 1u);
+    const uint32_t ball = __ballot_sync(0xffffffffu, mine);
+    if (mine) out[pos + __popc(ball & ((1u << lane) - 1u))] = j;
+    pos += __popc(ball);
+  }
+}
+
+}  // namespace rola
+
+using namespace rola;
+
+extern "C" size_t rola_select_workspace_bytes(const rola_shape_t* s) {
+  if (rola_internal::check_shape(s) != ROLA_OK) return 0;
+  const size_t nb = (size_t)rola_num_blocks(s);
+  const size_t pooled = 2 * (size_t)s->B * s->H * nb * s->d * sizeof(double);
+  const size_t scores = (size_t)s->B * s->H * nb * nb * sizeof(double);
+  return rola_internal::round_up(pooled, 256) + rola_internal::round_up(scores, 256);
+}
+
+extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_t* q,
+                                            const uint16_t* k, int32_t* idx, double* scores_opt,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  rola_status_t st = rola_internal::check_shape(s);
+  if (st != ROLA_OK) return st;
+  if (!q || !k || !idx) return ROLA_ERR_INVALID_ARG;
+  if (!rola_host::aligned(q, 16) || !rola_host::aligned(k, 16) || !rola_host::aligned(idx, 4) ||
+      (scores_opt && !rola_host::aligned(scores_opt, 8)))
+    return ROLA_ERR_ALIGNMENT;
+  const int nb = rola_num_blocks(s);
+  if (nb > 32 * kMaxPerLane) return ROLA_ERR_UNSUPPORTED;
+  const size_t need = rola_select_workspace_bytes(s);
+  if (!ws || ws_bytes < need || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  double* qbar = reinterpret_cast<double*>(ws);
+  double* kbar = qbar + (size_t)s->B * s->H * nb * s->d;
+  double* sig = reinterpret_cast<double*>(
+      reinterpret_cast<char*>(ws) +
+      rola_internal::round_up(2 * (size_t)s->B * s->H * nb * s->d * sizeof(double), 256));
+  if (scores_opt) sig = scores_opt;
+
+  pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
+  const int tiles = (nb + kScTile - 1) / kScTile;
+  score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, 0, cs>>>(qbar, kbar, sig, s->H, s->d, nb);
+  const int rows = s->B * s->H * nb;
+  topk_kernel<<<(rows + 7) / 8, 256, 0, cs>>>(sig, idx, rows, nb, s->k_b);
+  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+}

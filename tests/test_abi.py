@@ -1,0 +1,80 @@
+"""The C ABI: the library loads without a GPU, exports every entry point the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_linear_attention_mean_b200 import binding as rb
+from sparse_linear_attention_mean_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "rola.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return rb.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z][a-z0-9_]*)\s*\(", text)) - {"defined"})
+
+
+def test_header_declares_binding_exports():
+    assert declared_functions() == sorted(rb.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_kb_rule(lib):
+    for s in range(6):
+        assert lib.rola_status_string(s)
+    assert rb.kb_from_sparsity(100, 970) == 3
+    assert rb.kb_from_sparsity(591, 970) == 18
+    assert rb.kb_from_sparsity(256, 900) == 26
+    assert rb.kb_from_sparsity(16, 750) == 4
+    assert rb.kb_from_sparsity(0, 970) == -1
+    assert rb.kb_from_sparsity(10, 1000) == -1
+
+
+def test_num_blocks_and_workspace_sizes(lib):
+    s = rb.Shape(1, 40, 128, 21, 45, 80, 128, 18, 32)
+    assert rb.num_blocks(s) == 591
+    cs = s.c()
+    assert lib.rola_layer_workspace_bytes(ctypes.byref(cs)) > lib.rola_select_workspace_bytes(ctypes.byref(cs)) > 0
+    bad = rb.Shape(1, 40, 128, 21, 45, 80, 128, 592, 32).c()   # k_b > n_blocks
+    assert lib.rola_layer_workspace_bytes(ctypes.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("N", 123, 1),          # N != T*Hg*W
+    ("k_b", 0, 1),
+    ("k_b", 10_000, 1),
+    ("r", 3, 1),            # odd rank
+    ("d", 96, 2),           # valid but no kernel
+    ("block", 32, 2),
+    ("rope_base", -1.0, 1),
+])
+def test_bad_shapes_rejected_on_host(lib, field, value, status):
+    cs = rb.Shape(1, 2, 64, 4, 16, 16, 64, 4, 16).c()
+    setattr(cs, field, value)
+    dummy = ctypes.c_void_p(256)
+    st = lib.rola_block_states(ctypes.byref(cs), dummy, dummy, dummy, dummy, dummy, dummy, dummy, None)
+    assert st == status
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    cs = rb.Shape(1, 2, 64, 4, 16, 16, 64, 4, 16).c()
+    ok = ctypes.c_void_p(4096)
+    assert lib.rola_block_states(ctypes.byref(cs), None, ok, ok, ok, ok, ok, ok, None) == 1
+    odd = ctypes.c_void_p(4097)
+    assert lib.rola_block_states(ctypes.byref(cs), odd, ok, ok, ok, ok, ok, ok, None) == 5
+    assert lib.rola_select_blocks(ctypes.byref(cs), ok, ok, ok, None, None, 0, None) == 3  # no workspace
+    assert lib.fp8_quantize_rows_bf16(4, 15, ok, ok, ok, None) == 1                          # K % 16

@@ -1,0 +1,221 @@
+"""GPU parity of the RoLA path against the fp64 oracle, through the C ABI.
+
+* block masks: bit-exact; rows whose k-th and (k+1)-th scores lie within 1e-5
+  (relative) are reported and are the only rows allowed to differ;
+* states S_blk, z_blk, S, z: within 1e-4 relative (plus 1e-4 of the block's
+  largest magnitude);
+* attention output given the oracle's mask: |err| <= 1e-2 + 1e-2 |ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import rola_oracle as ro
+from sparse_linear_attention_mean_b200 import binding as rb
+from sparse_linear_attention_mean_b200 import synth
+
+from helpers import bf16_to_f64, check_close, dev_bf16, dev_inputs, mask_mismatch
+
+pytestmark = pytest.mark.gpu
+
+_CACHE = {}
+
+
+def workload_inputs(i):
+    if i not in _CACHE:
+        w = synth.WORKLOADS[i]
+        _CACHE.clear()
+        _CACHE[i] = (w, synth.make_inputs(w))
+    return _CACHE[i]
+
+
+def _grid(w):
+    return (w.T, w.Hg, w.W)
+
+
+def _states_check(w, inp, states, heads):
+    S_blk, z_blk, S_glb, z_glb = (t.cpu().numpy().astype(np.float64) for t in states)
+    for h in heads:
+        q, k, v, P = ro.head_slices(inp, 0, h)
+        th = ro.rope_angles(w.N, w.T, w.Hg, w.W, w.r, w.rope_base)
+        Sb, zb, S, z = ro.block_states(k, v, P, th, w.block)
+        scale = np.abs(Sb).max(axis=(1, 2), keepdims=True)
+        err = np.abs(S_blk[0, h] - Sb)
+        assert np.all(err <= 1e-4 * scale + 1e-4 * np.abs(Sb)), (h, float((err / (scale + 1e-30)).max()))
+        assert np.all(np.abs(z_blk[0, h] - zb) <= 1e-4 * np.abs(zb) + 1e-6), h
+        assert np.all(np.abs(S_glb[0, h] - S) <= 1e-4 * np.abs(S).max() + 1e-4 * np.abs(S)), h
+        assert np.all(np.abs(z_glb[0, h] - z) <= 1e-5 * np.abs(z)), h
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3])
+def test_select_blocks_bitexact(cfg):
+    w, inp = workload_inputs(cfg)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx_gpu, sc_gpu = rb.select_blocks(shape, q, k, scores=True)
+    idx_ref, sig = ro.select_all(inp, w.block, w.k_b)
+    idx_gpu = idx_gpu.cpu().numpy()
+    ties, bad = mask_mismatch(idx_gpu, idx_ref, sig, w.k_b)
+    assert not bad, f"mask rows differ outside near-ties: {bad[:5]}"
+    # scores agree to float64 rounding
+    np.testing.assert_allclose(sc_gpu.cpu().numpy(), sig, rtol=1e-12, atol=1e-12 * np.abs(sig).max())
+    n_ties = sum(len(ro.near_ties(sig[0, h], w.k_b)) for h in range(w.H))
+    print(f"workload {cfg}: {idx_ref.size // w.k_b} rows, near-tie rows {n_ties}, differing tie rows {len(ties)}")
+    # every row strictly ascending and in range
+    assert (np.diff(idx_gpu, axis=-1) > 0).all() and idx_gpu.min() >= 0 and idx_gpu.max() < w.n_blocks
+
+
+@pytest.mark.parametrize("cfg,heads", [(0, [0, 1]), (1, [0, 11]), (3, [0, 39])])
+def test_block_states(cfg, heads):
+    w, inp = workload_inputs(cfg)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    states = rb.block_states(shape, k, v, P)
+    torch.cuda.synchronize()
+    _states_check(w, inp, states, heads)
+
+
+def _attention_case(w, inp, heads, qblocks, gate_scale=1.0, idx_ref=None):
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    gate = gate * gate_scale
+    if idx_ref is None:
+        idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
+    idx = torch.from_numpy(idx_ref).cuda()
+    states = rb.block_states(shape, k, v, P)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = rb.attention_fwd(shape, q, k, v, idx, P, states, gate, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    o = bf16_to_f64(out)
+    inp2 = dict(inp)
+    inp2["gate"] = (inp["gate"].astype(np.float64) * gate_scale)
+    res = ro.rola_forward(inp2, bs=w.block, k_b=w.k_b, grid=_grid(w), rope_base=w.rope_base,
+                          idx=idx_ref, heads=heads, qblocks=qblocks)
+    worst = 0.0
+    for (b, h), r in res.items():
+        for a, rows in r.o.items():
+            lo, hi = ro.block_range(a, w.block, w.N)
+            worst = max(worst, check_close(o[b, lo:hi, h, :], rows, what=f"head {h} block {a}"))
+    return worst, out
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_attention_all_rows(cfg):
+    w, inp = workload_inputs(cfg)
+    worst, out = _attention_case(w, inp, heads=None, qblocks=None)
+    print(f"workload {cfg}: worst err/bound {worst:.3f}")
+    # padded rows are never written: the buffer beyond N does not exist, and
+    # every valid row is finite
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_attention_sampled(cfg):
+    w, inp = workload_inputs(cfg)
+    nb = w.n_blocks
+    qblocks = [0, 1, nb // 2, nb - 2, nb - 1]
+    worst, _ = _attention_case(w, inp, heads=[0, w.H - 1], qblocks=qblocks)
+    print(f"workload {cfg}: worst err/bound {worst:.3f}")
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_attention_linear_branch_dominant(cfg):
+    # o_lin of zero-mean v is ~1e-3; a gate of 1e3 makes the linear branch
+    # carry the output so that its parity is visible at the same tolerance.
+    w, inp = workload_inputs(cfg)
+    worst, _ = _attention_case(w, inp, heads=[0, w.H - 1], qblocks=None, gate_scale=1000.0)
+    print(f"workload {cfg} gate x1000: worst err/bound {worst:.3f}")
+
+
+def test_attention_gate_zero_is_block_sparse():
+    w = synth.custom_workload(synth.WORKLOADS[0], gate_const=0.0)
+    inp = synth.make_inputs(w)
+    worst, _ = _attention_case(w, inp, heads=None, qblocks=None)
+
+
+@pytest.mark.parametrize("T,Hg,W,block,d,r,kb", [
+    (2, 8, 9, 64, 64, 16, 3),      # 144 tokens: ragged last block of 16
+    (3, 5, 7, 64, 64, 32, 1),      # 105 tokens, one kept block
+    (2, 8, 9, 128, 128, 32, 2),    # 2 blocks of 128, last has 16 valid
+    (3, 9, 10, 128, 64, 16, 2),    # d = 64 with 128-token blocks
+])
+def test_attention_ragged_small(T, Hg, W, block, d, r, kb):
+    w = synth.Workload("ragged", 1, 3, d, T, Hg, W, block, 0, kb, r, seed=7)
+    inp = synth.make_inputs(w)
+    worst, _ = _attention_case(w, inp, heads=None, qblocks=None)
+    worst_l, _ = _attention_case(w, inp, heads=None, qblocks=None, gate_scale=1000.0)
+
+
+@pytest.mark.parametrize("block,d,r", [(64, 64, 16), (128, 128, 32)])
+def test_dense_limit_s0(block, d, r):
+    T, Hg, W = (2, 8, 16) if block == 64 else (2, 16, 20)
+    N = T * Hg * W
+    nb = -(-N // block)
+    w = synth.Workload("dense", 1, 2, d, T, Hg, W, block, 0, nb, r, seed=11)
+    inp = synth.make_inputs(w)
+    worst, out = _attention_case(w, inp, heads=None, qblocks=None, gate_scale=1000.0)
+    # with every block kept, o_lin is exactly 0: the output is plain softmax attention
+    q, k, v = (torch.from_numpy(ro.bf16_to_f64(inp[x])).permute(0, 2, 1, 3) for x in ("q", "k", "v"))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v).permute(0, 2, 1, 3).numpy()
+    check_close(bf16_to_f64(out), ref, what="dense limit vs SDPA")
+
+
+def test_batch_two_matches_single():
+    w = synth.custom_workload(synth.WORKLOADS[0], B=2)
+    inp = synth.make_inputs(w)
+    idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx_gpu = rb.select_blocks(shape, q, k).cpu().numpy()
+    assert np.array_equal(idx_gpu, idx_ref)
+    _attention_case(w, inp, heads=None, qblocks=None)
+
+
+def test_bad_index_reported_not_trapped():
+    w, inp = workload_inputs(0)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
+    bad = idx_ref.copy()
+    bad[0, 0, 3, 1] = 999            # out of range
+    bad[0, 1, 5, 2] = bad[0, 1, 5, 1]  # duplicate (not ascending)
+    states = rb.block_states(shape, k, v, P)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = rb.attention_fwd(shape, q, k, v, torch.from_numpy(bad).cuda(), P, states, gate, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & rb.DEVERR_BAD_INDEX
+    assert not (int(err.item()) & rb.DEVERR_TIMEOUT)
+    # untouched rows still match the oracle
+    o = bf16_to_f64(out)
+    res = ro.rola_forward(inp, bs=w.block, k_b=w.k_b, grid=_grid(w), idx=idx_ref, heads=[0], qblocks=[0, 1])
+    for a, rows in res[(0, 0)].o.items():
+        lo, hi = ro.block_range(a, w.block, w.N)
+        check_close(o[0, lo:hi, 0, :], rows)
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_layer_entry_points(cfg):
+    w, inp = workload_inputs(cfg)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx = torch.empty((1, w.H, w.n_blocks, w.k_b), dtype=torch.int32, device="cuda")
+    layer = rb.Layer(shape)
+    out = layer(q, k, v, P, gate, idx_out=idx)
+    torch.cuda.synchronize()
+    assert int(layer.dev_err.item()) == 0
+    idx_ref, sig = ro.select_all(inp, w.block, w.k_b)
+    ties, bad = mask_mismatch(idx.cpu().numpy(), idx_ref, sig, w.k_b)
+    assert not bad
+    # same as the three calls in sequence
+    idx2 = rb.select_blocks(shape, q, k)
+    out2 = rb.attention_fwd(shape, q, k, v, idx2, P, rb.block_states(shape, k, v, P), gate)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    # host-buffer variant: pinned host tensors in, host tensor out
+    host = [t.cpu().pin_memory() for t in (q, k, v, P, gate)]
+    out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    hl = rb.HostLayer(shape)
+    hl(*host, out_h)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, out.cpu())
