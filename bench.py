@@ -1,0 +1,361 @@
+"""Benchmark of the RoLA attention layer on B200.
+
+One step = one RoLA attention layer (block selection, linear-branch states,
+fused sparse + linear attention) over the Wan2.1-14B 720P attention shape at
+97 % block sparsity: B=1, H=40, d=128, 21x45x80 latent grid (N=75600 tokens,
+591 blocks of 128, 18 kept per query block), rank 32.  Inputs are the seeded
+synthetic tensors of ``synth`` (2.3 GB of q/k/v, larger than the 126 MB L2,
+so no flush is needed between steps).
+
+Printed (rank 0, one JSON line): effective TFLOP/s over the computed blocks
+(4 * 128^2 * d per kept block pair, QK^T and PV) for the whole job, ms per
+layer, per-kernel times, the roofline of the dominant kernel, an end-to-end
+figure through the host-buffer entry point, the fp64 oracle timed on the host
+cores on a bounded sample, and the SM clocks seen during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (under torchrun) every rank runs an independent replica of the
+layer; the whole-job figure is N x work / (max over ranks of the time).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "RoLA attn fwd ms/layer & effective TFLOPS (% B200 BF16 peak), Wan-14B 720P 97%"
+UNIT = "TFLOP/s"
+WORKLOAD_ID = 3
+
+
+def workload_config(w) -> dict:
+    return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d,
+            "grid_thw": [w.T, w.Hg, w.W], "N": w.N, "block": w.block,
+            "n_blocks": w.n_blocks, "sparsity_permille": w.sparsity_permille, "k_b": w.k_b,
+            "rank": w.r, "flop_per_layer": w.sparse_flops(),
+            "l2": "inputs 2.3 GB > 126 MB L2, no flush between steps"}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self) -> dict | None:
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, x in enumerate(fl) if x.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, inp, heads=(0,), qblocks=None):
+    """Runs the fp64 oracle on a bounded sample; returns (seconds, flop, text)."""
+    from oracle import rola_oracle as ro
+    nb = w.n_blocks
+    qb = list(range(nb)) if qblocks is None else list(qblocks)
+    t0 = time.perf_counter()
+    ro.rola_forward(inp, bs=w.block, k_b=w.k_b, grid=(w.T, w.Hg, w.W), rope_base=w.rope_base,
+                    heads=list(heads), qblocks=qb)
+    dt = time.perf_counter() - t0
+    flop = 4.0 * w.block * w.block * w.d * w.k_b * len(qb) * len(heads)
+    text = (f"fp64 oracle on {len(heads)} head(s) x {len(qb)} of {nb} query blocks "
+            f"(selection and states over the whole head included)")
+    return dt, flop, text
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w, inp) -> dict:
+    dt, flop, text = oracle_sample(w, inp, heads=(0,), qblocks=range(0, w.n_blocks, 4))
+    return {"value": flop / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": text + f"; {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args) -> int:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from sparse_linear_attention_mean_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    inp = synth.make_inputs(w)
+    qblocks = range(0, w.n_blocks, 8)     # bounded sample per step: 74 query blocks of one head
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, heads=(0,), qblocks=qblocks)
+    times, flop, text = [], 0.0, ""
+    for s in range(args.steps):
+        dt, flop, text = oracle_sample(w, inp, heads=(s % w.H,), qblocks=qblocks)
+        times.append(dt)
+    tot = sum(times)
+    value = flop * len(times) / tot / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": text + " per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    from sparse_linear_attention_mean_b200 import binding as rb
+    from sparse_linear_attention_mean_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    w = synth.WORKLOADS[args.workload]
+    shape = rb.Shape.of(w)
+    inp = synth.make_inputs(w)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+    q, k, v, P = dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["P"])
+    gate = torch.from_numpy(inp["gate"]).cuda()
+    stream = torch.cuda.current_stream()
+
+    # persistent buffers for the three stages (the layer's own workspace layout)
+    nb = w.n_blocks
+    idx = torch.empty((w.B, w.H, nb, w.k_b), dtype=torch.int32, device="cuda")
+    S_blk = torch.empty((w.B, w.H, nb, w.r, w.d), dtype=torch.float32, device="cuda")
+    z_blk = torch.empty((w.B, w.H, nb, w.r), dtype=torch.float32, device="cuda")
+    S_glb = torch.empty((w.B, w.H, w.r, w.d), dtype=torch.float32, device="cuda")
+    z_glb = torch.empty((w.B, w.H, w.r), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device="cuda")
+    dev_err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    import ctypes
+    L = rb.lib()
+    cs = shape.c()
+    sel_ws_bytes = L.rola_select_workspace_bytes(ctypes.byref(cs))
+    sel_ws = torch.empty(sel_ws_bytes, dtype=torch.uint8, device="cuda")
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    P_ = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def select():
+        st = L.rola_select_blocks(ctypes.byref(cs), P_(q), P_(k), P_(idx), None, P_(sel_ws),
+                                  sel_ws_bytes, sptr)
+        assert st == 0, st
+
+    def states():
+        st = L.rola_block_states(ctypes.byref(cs), P_(k), P_(v), P_(P), P_(S_blk), P_(z_blk),
+                                 P_(S_glb), P_(z_glb), sptr)
+        assert st == 0, st
+
+    def attention():
+        st = L.rola_attention_fwd(ctypes.byref(cs), P_(q), P_(k), P_(v), P_(idx), P_(P), P_(S_blk),
+                                  P_(z_blk), P_(S_glb), P_(z_glb), P_(gate), P_(out), P_(dev_err), sptr)
+        assert st == 0, st
+
+    stages = [("select", select, 3), ("states", states, 2), ("attention", attention, 1)]
+    for _ in range(args.warmup):
+        for _, fn, _ in stages:
+            fn()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        for s in range(K):
+            ev[s][0].record(stream)
+            for i, (_, fn, _) in enumerate(stages):
+                fn()
+                ev[s][i + 1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    assert int(dev_err.item()) == 0, f"device error flag {int(dev_err.item())}"
+
+    per_stage = {nm: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)]
+                 for i, (nm, _, _) in enumerate(stages)}
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][len(stages)])
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / K
+    flop = w.sparse_flops()
+    value = world * flop * K / (total_ms * 1e-3) / 1e12
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        host = [x.cpu().pin_memory() for x in (q, k, v, P, gate)]
+        out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+        hl = rb.HostLayer(shape)
+        for _ in range(max(1, args.warmup)):
+            hl(*host, out_h)
+        torch.cuda.synchronize()
+        K2 = max(2, min(K, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K2):
+            hl(*host, out_h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / K2
+        t2 = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t2.item())
+        e2e = {"value": world * flop / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
+               "d2h_bytes_per_step": out_h.numel() * out_h.element_size()}
+
+    if rank == 0:
+        peaks = measured_peaks()
+        att_ms = statistics.mean(per_stage["attention"])
+        achieved = flop / (att_ms * 1e-3) / 1e12
+        traffic = None
+        prof = os.path.join(ROOT, "profiles", "attention_traffic.json")
+        if os.path.exists(prof):
+            with open(prof) as f:
+                tr = json.load(f)
+            if tr.get("kernel_hash") == kernel_hash():
+                traffic = tr.get("bytes_per_launch")
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**workload_config(w), "parallelism": f"replicas x{world}"},
+            "kernels_ms": {nm: statistics.mean(x) for nm, x in per_stage.items()},
+            "attention_tflops": achieved,
+            "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
+            "roofline": {"bound": "tensor", "kernel": "rola_attn_kernel", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                         "peak_source": peaks["source"] + " bf16 burst"},
+            "e2e": e2e,
+            "gpu_launches": K * sum(n for _, _, n in stages),
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, inp)
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for nm in ("rola_attention.cu", "rola_common.cuh"):
+        with open(os.path.join(ROOT, "sparse_linear_attention_mean_b200", "csrc", nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling runs)")
+    ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
+                    help="attention workload id of synth.WORKLOADS (profiling of smaller cases)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
