@@ -583,6 +583,15 @@ static rola_status_t launch_attn(const rola_shape_t* s, const uint16_t* q, const
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 
+// The persistent two-tile kernel (rola_attention_pair.cu) serves d = 128 with
+// 128-token blocks and k_b <= 256; this one-tile kernel serves the rest.
+bool pair_kernel_supports(const rola_shape_t* s);
+rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const int32_t* idx, const uint16_t* P,
+                                 const float* S_blk, const float* z_blk, const float* S_glb,
+                                 const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
+                                 cudaStream_t cs);
+
 }  // namespace rola
 
 using namespace rola;
@@ -622,6 +631,8 @@ extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_
   prm.dev_err = dev_err;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (pair_kernel_supports(s))
+    return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, cs);
   if (s->d == 128 && s->block == 128 && s->r == 32) return launch_attn<128, 128, 32>(s, q, k, v, prm, cs);
   if (s->d == 128 && s->block == 128 && s->r == 16) return launch_attn<128, 128, 16>(s, q, k, v, prm, cs);
   if (s->d == 64 && s->block == 64 && s->r == 16) return launch_attn<64, 64, 16>(s, q, k, v, prm, cs);

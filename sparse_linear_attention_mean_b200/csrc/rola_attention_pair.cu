@@ -1,0 +1,828 @@
+// RoLA attention forward, persistent two-tile kernel for 128-token blocks and
+// d = 128 (the Wan attention shapes).
+//
+// SparkDiffusion write-up (0539edu.com news page), section 05: the sparse
+// branch keeps the high-energy query-key blocks, a rotary low-rank linear
+// branch restores the dropped context; section 01: at 97 % sparsity only 3 %
+// of the blocks remain, so the kernel must turn few, scattered blocks into
+// dense tensor-core work.
+//
+// A CTA is persistent and works on units: two adjacent query blocks
+// (2p, 2p+1) of one (batch, head), one per slot.  Their kept lists overlap
+// heavily, so the CTA walks the ascending UNION of both lists; each key block
+// is loaded once (TMA, gathered by block index) and multiplied by the query
+// tile of every slot that keeps it.  Tensor memory holds S0, S1, O0, O1
+// (4 x 128 columns); the bf16 probabilities P overwrite the first 64 columns
+// of their S buffer and feed P.V straight from tensor memory.
+//
+// Warp roles (12 warps, three warpgroups):
+//   warps 0-3, 4-7  one slot each (184 registers): softmax -- thread i owns
+//                   query row i, loads its 128 scores with one tensor-memory
+//                   read, and rescales O lazily (only when the row max grows
+//                   by more than 2^8, which keeps P <= 256); at the tile end
+//                   rho_q = R(t, y, x) phi(q P_h) (rotary angles from a per-CTA
+//                   cos/sin table), psi_q . z_U, and the epilogue
+//                   o = O / l + g_h * L / (psi_q . z_U)
+//   warp 8          producer: unit lists, Q tiles, K/V ring (TMA)
+//   warp 9          MMA issuer: S = Q K^T, O += P V, q P_h, L = rho_q S_U
+//   warps 10-11     head projection P_h^T to shared memory; gather of the
+//                   linear-branch states of every union block into fp32
+//                   shared-memory accumulators; S_U = S - sum_kept S_j, z_U
+// The linear branch is folded into O: at a tile end the softmax warps write
+// rho'_q = rho_q g_h l / (psi_q . z_U) (bf16 hi + lo) into tensor memory and
+// one more MMA adds rho'_q S_U to O, S_U coming from the gather warps'
+// accumulators converted in place; the epilogue is then out = O / l.  The
+// next unit's S MMAs do not wait for that epilogue, only its first P.V does.
+// Every wait is bounded; on a timeout the CTA drains its copies and MMAs,
+// frees tensor memory and reports ROLA_DEVERR_TIMEOUT.
+#include <math.h>
+
+#include "rola_common.cuh"
+#include "rola_internal.h"
+
+namespace rola {
+namespace pairk {
+
+constexpr int kThreads = 384;
+constexpr int kMaxKept = 256;           // k_b limit of this kernel
+constexpr int kMaxUnion = 2 * kMaxKept;
+constexpr int NR = 3;                   // K/V ring slots (each one K or one V tile)
+constexpr int D = 128, BM = 128, BN = 128;
+constexpr uint32_t TILE = BM * D * 2;   // 32 KB: one Q, K or V tile
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+// Moving every kEmuEvery-th exp2 pair onto the FMA pipe (exp2_poly2) was
+// measured slower on B200 for this kernel (the softmax is not bound by the
+// special-function unit), so it is off.
+constexpr bool kEmuExp2 = false;
+constexpr int kEmuEvery = 4;
+
+template <int R>
+struct Layout {
+  static constexpr uint32_t q_off = 0;                    // 2 tiles
+  static constexpr uint32_t ring_off = q_off + 2 * TILE;  // NR tiles
+  static constexpr uint32_t pt_off = ring_off + NR * TILE;
+  static constexpr uint32_t PT_BYTES = 32 * D * 2;
+  static constexpr uint32_t acc_off = pt_off + PT_BYTES;  // fp32 state accumulators [2][r * d]
+  static constexpr uint32_t misc_off = (acc_off + 2 * R * D * 4 + 1023) / 1024 * 1024;
+  // S_U (bf16 hi, then lo) replaces a slot's accumulator in place
+  static constexpr uint32_t SU_BYTES = R * D * 2;
+  static_assert(acc_off % 1024 == 0 && (R * D * 4) % 1024 == 0, "S_U operands need 1024-byte alignment");
+  // tensor memory columns
+  // S_s at columns [128 s, 128 s + 128), O_s at [256 + 128 s, ...): s_col / o_col
+
+  static constexpr uint32_t P_OFF = 0;  // bf16 P over the first 64 columns of its S buffer
+};
+
+struct UnitList {
+  int b, h, a[2];
+  int active[2];
+  int nu;
+  int cnt[2];
+  int lin_empty[2];
+  int raw[2][kMaxKept];
+  int ulist[kMaxUnion];
+  uint8_t umask[kMaxUnion];
+};
+
+constexpr int kTabCap = 1024;  // cos/sin entries of the rotary table in shared memory
+
+struct Misc {
+  uint64_t list_full[2], list_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t ring_full[NR], ring_empty[NR];
+  uint64_t s_full[2], p_full[2];
+  uint64_t pt_full, qt_full[2], zu_ready[2], cvt[2], lin_ready[2], l_done[2], o_free[2];
+  uint64_t mma_final;
+  uint32_t tmem_base;
+  int abort;
+  int err;
+  float zU[2][32];
+  float2 tab[kTabCap];  // (cos, sin) of pos * freq per rotation pair and grid position
+  UnitList L[2];
+};
+
+struct Params {
+  int B, H, N, nb, kb, T, Hg, W, npairs, units;
+  float scale_log2;
+  const int32_t* idx;
+  const uint16_t* P;
+  const float* S_blk;
+  const float* z_blk;
+  const float* S_glb;
+  const float* z_glb;
+  const float* gate;
+  uint16_t* out;
+  int32_t* dev_err;
+  RopeTable rope;
+  // rotary table: entry of pair pr at position pos = tab_base[pr] + pos * tab_stride[pr];
+  // pair pr fills entries [tab_first[pr], tab_first[pr + 1]) of the fill order
+  int tab_base[16], tab_stride[16], tab_first[17];
+  int tab_entries;
+};
+
+ROLA_DEV uint32_t s_col(int s) { return (uint32_t)s * 128u; }
+ROLA_DEV uint32_t o_col(int s) { return 256u + (uint32_t)s * 128u; }
+
+ROLA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+ROLA_DEV uint64_t desc_k_sw128(uint32_t base, int rows, int kk) {
+  return smem_desc(base + (uint32_t)(kk >> 2) * rows * 128 + (uint32_t)(kk & 3) * 32, 16, 1024,
+                   kSwizzle128B);
+}
+// Descriptor of k-step kk from the descriptor of k-step 0: only the start
+// address field (bits 0-13, in 16-byte units) moves, and shared-memory
+// addresses stay below 2^18 bytes, so a plain add cannot carry out of it.
+ROLA_DEV constexpr uint64_t kstep_k_sw128(int rows, int kk) {
+  return (uint64_t)(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
+}
+template <uint32_t N>
+ROLA_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+ROLA_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
+ROLA_DEV void decode_unit(const Params& p, int id, int& b, int& h, int& pair) {
+  pair = id % p.npairs;
+  h = (id / p.npairs) % p.H;
+  b = id / (p.npairs * p.H);
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    rola_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using Ly = Layout<R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& M = *reinterpret_cast<Misc*>(smem + Ly::misc_off);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (p.dev_err && (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)) return;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&M.list_full[i], 1);
+      mbar_init(&M.list_empty[i], 1 + 2 * 128 + 64);
+      mbar_init(&M.q_full[i], 1);
+      mbar_init(&M.q_empty[i], 1);
+      mbar_init(&M.s_full[i], 1);
+      mbar_init(&M.p_full[i], 128);
+      mbar_init(&M.qt_full[i], 1);
+      mbar_init(&M.zu_ready[i], 64);
+      mbar_init(&M.cvt[i], 64);
+      mbar_init(&M.lin_ready[i], 128);
+      mbar_init(&M.l_done[i], 1);
+      mbar_init(&M.o_free[i], 128);
+    }
+    for (int i = 0; i < NR; ++i) {
+      mbar_init(&M.ring_full[i], 1);
+      mbar_init(&M.ring_empty[i], 1);
+    }
+    mbar_init(&M.pt_full, 64);
+    mbar_init(&M.mma_final, 1);
+    M.abort = 0;
+    M.err = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&M.tmem_base, 512);
+    tmem_relinquish();
+  }
+  // rotary cos/sin table, once per (persistent) CTA
+  for (int e = tid; e < p.tab_entries; e += kThreads) {
+    int pr = 0;
+    while (pr + 1 < R / 2 && e >= p.tab_first[pr + 1]) ++pr;
+    const int pos = e - p.tab_first[pr];
+    float sn, cs;
+    rope_sincos(pos, p.rope.freq[pr], &sn, &cs);
+    M.tab[p.tab_base[pr] + pos * p.tab_stride[pr]] = make_float2(cs, sn);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = M.tmem_base;
+  volatile int* abort = &M.abort;
+  const int my_units = p.units > (int)blockIdx.x ? (p.units - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp < 8) {
+    // ================================================================ one slot: softmax, rho_q, epilogue
+    setmaxnreg_inc<184>();
+    const int s = warp >> 2;
+    const int row = tid & 127;
+    const uint32_t trow = tm + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t sc = trow + s_col(s);
+    const uint32_t oc = trow + o_col(s);
+    const uint64_t sc2 = f32x2(p.scale_log2, p.scale_log2);
+    uint32_t nsc = 0, uc = 0;
+    bool ok = true;
+    for (int u = 0; ok && u < my_units; ++u) {
+      const int buf = u & 1;
+      if (!(ok = warp_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+      const UnitList& U = M.L[buf];
+      if (U.active[s]) {
+        float m = 0.f, l = 0.f;
+        bool first = true;
+        for (int j = 0; j < U.nu; ++j) {
+          if (!((U.umask[j] >> s) & 1)) continue;
+          if (!(ok = warp_wait(&M.s_full[s], nsc & 1, abort))) break;
+          ++nsc;
+          tc_fence_after();
+          uint32_t x[128];
+          tmem_ld32_at<0>(sc, x);
+          tmem_ld32_at<32>(sc + 32, x);
+          tmem_ld32_at<64>(sc + 64, x);
+          tmem_ld32_at<96>(sc + 96, x);
+          tmem_wait_ld();
+          const int blk = U.ulist[j];
+          if (blk == p.nb - 1) {
+            // padded keys of the last block take no part in the softmax
+            const int valid = p.N - blk * BN;
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= valid) x[c] = __float_as_uint(-INFINITY);
+          }
+          float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 128; c += 4) {
+            m0 = fmax3(m0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+            m1 = fmax3(m1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+          }
+          // lazy rescaling: the exponent base m moves only when the row max
+          // exceeds it by more than 2^8 (P then stays <= 256)
+          const float mc = fmaxf(m0, m1) * p.scale_log2;
+          float alpha = 1.f;
+          bool need = false;
+          if (first) {
+            m = mc;
+          } else if (mc > m + kRescaleThreshold) {
+            need = true;
+            alpha = fast_exp2(m - mc);
+            m = mc;
+          }
+          const uint64_t nm2 = f32x2(-m, -m);
+          uint64_t acc2 = f32x2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            float y0, y1, p0, p1;
+            f32x2_split(ffma2(f32x2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2, nm2), y0, y1);
+            if (kEmuExp2 && (c >> 1) % kEmuEvery == kEmuEvery - 1) {
+              exp2_poly2(y0, y1, p0, p1);  // FMA pipe
+            } else {
+              p0 = fast_exp2(y0);          // special-function unit
+              p1 = fast_exp2(y1);
+            }
+            acc2 = fadd2(acc2, f32x2(p0, p1));
+            x[c >> 1] = pack_bf16(p0, p1);
+          }
+          // bf16 P over columns [0, 64) of the S buffer (S already read)
+          tmem_st32_at<0>(sc + Ly::P_OFF, x);
+          tmem_st32_at<32>(sc + Ly::P_OFF + 32, x);
+          float s0, s1;
+          f32x2_split(acc2, s0, s1);
+          l = l * alpha + (s0 + s1);
+          first = false;
+          if (__any_sync(0xffffffffu, need)) {
+            // O holds the previous P.V, complete because that MMA was issued
+            // before this S; the next P.V waits for p_full.
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(oc + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(oc + c * 32, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&M.p_full[s]);
+        }
+        if (!ok) break;
+        // ---- tile end.  The linear branch is folded into O:
+        //   O += rho'_q S_U,  rho'_q = rho_q * g_h * l / (psi_q . z_U),
+        // so that the epilogue is out = O / l.  rho'_q (bf16 hi + lo) goes to
+        // columns [32, 32 + r) of this slot's S buffer as the A operand of
+        // that MMA; q P_h sits in columns [0, r).
+        if (!(ok = warp_wait(&M.qt_full[s], uc & 1, abort))) break;
+        tc_fence_after();
+        uint32_t qt[32];
+        if constexpr (R == 32) {
+          tmem_ld32(sc, qt);
+        } else {
+          tmem_ld16(sc, *reinterpret_cast<uint32_t(*)[16]>(&qt[0]));
+        }
+        tmem_wait_ld();
+        const int n = U.a[s] * BM + row;
+        const int nn = n < p.N ? n : p.N - 1;
+        const int pt_ = nn / (p.Hg * p.W), py = (nn / p.W) % p.Hg, px = nn % p.W;
+        float2 cs[R / 2];
+#pragma unroll
+        for (int pr = 0; pr < R / 2; ++pr) {
+          const int ax = p.rope.axis[pr];
+          cs[pr] = M.tab[p.tab_base[pr] + (ax == 0 ? pt_ : (ax == 1 ? py : px)) * p.tab_stride[pr]];
+        }
+#pragma unroll
+        for (int c = 0; c < R; ++c) qt[c] = __float_as_uint(phi(__uint_as_float(qt[c])));  // psi_q
+        if (!(ok = warp_wait(&M.zu_ready[s], uc & 1, abort))) break;
+        float den = 0.f;
+#pragma unroll
+        for (int c = 0; c < R; ++c) den = fmaf(__uint_as_float(qt[c]), M.zU[s][c], den);
+        const bool have_o = U.cnt[s] > 0;
+        const float lsum = have_o ? l : 1.f;
+        const float scale = U.lin_empty[s] ? 0.f : p.gate[U.h] * lsum / den;
+        uint32_t rh[R / 2], rl[R / 2];
+#pragma unroll
+        for (int pr = 0; pr < R / 2; ++pr) {
+          const float x0 = __uint_as_float(qt[2 * pr]), x1 = __uint_as_float(qt[2 * pr + 1]);
+          const float r0 = (x0 * cs[pr].x - x1 * cs[pr].y) * scale;
+          const float r1 = (x0 * cs[pr].y + x1 * cs[pr].x) * scale;
+          rh[pr] = pack_bf16(r0, r1);
+          rl[pr] = pack_bf16(r0 - bf16_lo(rh[pr]), r1 - bf16_hi(rh[pr]));
+        }
+        if constexpr (R == 32) {
+          tmem_st16(sc + 32, rh);
+          tmem_st16(sc + 48, rl);
+        } else {
+          tmem_st8(sc + 32, rh);
+          tmem_st8(sc + 40, rl);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&M.lin_ready[s]);
+        // ---- epilogue: out = O / l
+        if (!(ok = warp_wait(&M.l_done[s], uc & 1, abort))) break;
+        tc_fence_after();
+        const float inv_l = 1.f / lsum;
+        const bool write = n < p.N;
+        uint16_t* orow = p.out + (((size_t)U.b * p.N + (write ? n : 0)) * p.H + U.h) * D;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t o[64];
+          tmem_ld32_at<0>(oc + hf * 64, o);
+          tmem_ld32_at<32>(oc + hf * 64 + 32, o);
+          tmem_wait_ld();
+          uint32_t wv[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+          if (write) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + hf * 64);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&M.o_free[s]);
+        ++uc;
+      }
+      mbar_arrive(&M.list_empty[buf]);
+    }
+  } else {
+    setmaxnreg_dec<136>();
+    if (warp >= 10) {
+      // ============================================================== P_h, state gather, S_U
+      // acc[s] starts as the global state S and loses the state of every
+      // block slot s keeps, so it ends as S_U = S - sum_kept S_j; it is then
+      // converted in place into the bf16 hi + lo MN-major B operand of the
+      // linear-branch MMA (N = d, K = r, 128-byte swizzle).
+      const int t = tid - 320;  // 0..63
+      constexpr int PER = R * D / 256;  // float4 of a block state per thread
+      float4* accs = reinterpret_cast<float4*>(smem + Ly::acc_off);  // [2][R*D/4]
+      uint32_t uc[2] = {0, 0};
+      bool ok = true;
+      for (int u = 0; ok && u < my_units; ++u) {
+        const int buf = u & 1;
+        if (!(ok = warp_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+        const UnitList& U = M.L[buf];
+        const int b = U.b, h = U.h;
+        const size_t bh = (size_t)b * p.H + h;
+        // the previous unit's linear-branch MMAs read these accumulators
+        // (and its q P_h MMAs read P_h^T) -- wait for them
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (ok && uc[s] >= 1) ok = warp_wait(&M.l_done[s], (uc[s] - 1) & 1, abort);
+        if (!ok) break;
+        // P_h^T (K-major, N = r rows, K = d, 128-byte swizzle)
+        {
+          uint8_t* pt = smem + Ly::pt_off;
+          for (int e = t; e < R * D; e += 64) {
+            const int c = e / R, rr = e % R;
+            const uint16_t val = p.P[((size_t)h * D + c) * R + rr];
+            const int byte = (c & 63) * 2;
+            const int chunk = (byte >> 4) ^ (rr & 7);
+            *reinterpret_cast<uint16_t*>(pt + (c >> 6) * (32 * 128) + rr * 128 + chunk * 16 + (byte & 15)) = val;
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&M.pt_full);
+        }
+        // each thread owns float4 entries t + 64 i of both accumulators
+        {
+          const float4* Sg = reinterpret_cast<const float4*>(p.S_glb + bh * R * D);
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            const float4 g4 = __ldg(Sg + t + 64 * i);
+            accs[t + 64 * i] = g4;
+            accs[R * D / 4 + t + 64 * i] = g4;
+          }
+        }
+        const float zg = t < R ? p.z_glb[bh * R + t] : 0.f;
+        float zs[2] = {zg, zg};
+        for (int j = 0; j < U.nu; ++j) {
+          const size_t st = bh * p.nb + U.ulist[j];
+          const float4* src = reinterpret_cast<const float4*>(p.S_blk + st * R * D);
+          const int mk = U.umask[j];
+          float4 xv[PER];
+#pragma unroll
+          for (int i = 0; i < PER; ++i) xv[i] = __ldg(src + t + 64 * i);
+          const float zv = t < R ? __ldg(p.z_blk + st * R + t) : 0.f;
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            if (!((mk >> sl) & 1)) continue;
+            float4* a = accs + sl * (R * D / 4);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+              float4 v = a[t + 64 * i];
+              v.x -= xv[i].x;
+              v.y -= xv[i].y;
+              v.z -= xv[i].z;
+              v.w -= xv[i].w;
+              a[t + 64 * i] = v;
+            }
+            zs[sl] -= zv;
+          }
+        }
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (!ok || !U.active[s]) continue;
+          float4* a = accs + s * (R * D / 4);
+          float4 v[PER];
+#pragma unroll
+          for (int i = 0; i < PER; ++i) v[i] = a[t + 64 * i];
+          // every thread has read its part before anyone overwrites the region
+          mbar_arrive(&M.cvt[s]);
+          if (!(ok = warp_wait(&M.cvt[s], uc[s] & 1, abort))) continue;
+          uint8_t* su_hi = reinterpret_cast<uint8_t*>(a);
+          uint8_t* su_lo = su_hi + Ly::SU_BYTES;
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            const uint32_t h01 = pack_bf16(v[i].x, v[i].y), h23 = pack_bf16(v[i].z, v[i].w);
+            const uint32_t l01 = pack_bf16(v[i].x - bf16_lo(h01), v[i].y - bf16_hi(h01));
+            const uint32_t l23 = pack_bf16(v[i].z - bf16_lo(h23), v[i].w - bf16_hi(h23));
+            const int f = (t + 64 * i) * 4;
+            const int c = f / D, e = f % D;
+            const uint32_t off = (e >> 6) * (R * 128) + (c >> 3) * 1024 + (c & 7) * 128 +
+                                 ((((e & 63) >> 3) ^ (c & 7)) << 4) + (e & 7) * 2;
+            *reinterpret_cast<uint2*>(su_hi + off) = make_uint2(h01, h23);
+            *reinterpret_cast<uint2*>(su_lo + off) = make_uint2(l01, l23);
+          }
+          if (t < R) M.zU[s][t] = zs[s];
+          fence_proxy_async_smem();
+          mbar_arrive(&M.zu_ready[s]);
+          ++uc[s];
+        }
+        if (!ok) break;
+        mbar_arrive(&M.list_empty[buf]);
+      }
+    } else if (warp == 8) {
+      // ================================================================ producer
+      uint32_t g = 0, uc[2] = {0, 0};
+      int ring_par[NR], q_par[2] = {-1, -1};
+      for (int i = 0; i < NR; ++i) ring_par[i] = -1;
+      bool ok = true;
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+      }
+      for (int u = 0; ok && u < my_units; ++u) {
+        const int buf = u & 1;
+        if (u >= 2 && !(ok = warp_wait(&M.list_empty[buf], ((u >> 1) - 1) & 1, abort))) break;
+        UnitList& U = M.L[buf];
+        int b, h, pair;
+        decode_unit(p, (int)blockIdx.x + u * (int)gridDim.x, b, h, pair);
+        const int a0 = 2 * pair, a1 = 2 * pair + 1;
+        const size_t bh = (size_t)b * p.H + h;
+        for (int i = lane; i < 2 * p.kb; i += 32) {
+          const int s = i / p.kb, a = s ? a1 : a0;
+          U.raw[s][i % p.kb] = a < p.nb ? p.idx[(bh * p.nb + a) * p.kb + i % p.kb] : -1;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          // Validate both kept lists (in range, strictly ascending; a bad
+          // entry is skipped and reported) and merge them into one ascending
+          // union with a per-slot membership mask.
+          U.b = b;
+          U.h = h;
+          U.a[0] = a0;
+          U.a[1] = a1;
+          U.active[0] = a0 < p.nb;
+          U.active[1] = a1 < p.nb;
+          int pos[2] = {0, 0}, prev[2] = {-1, -1}, len[2];
+          len[0] = U.active[0] ? p.kb : 0;
+          len[1] = U.active[1] ? p.kb : 0;
+          U.cnt[0] = U.cnt[1] = 0;
+          int nu = 0, err = 0;
+          while (true) {
+            int best = 0x7fffffff;
+            for (int s = 0; s < 2; ++s) {
+              while (pos[s] < len[s]) {
+                const int v = U.raw[s][pos[s]];
+                if (v < 0 || v >= p.nb || v <= prev[s]) { err = 1; ++pos[s]; continue; }
+                break;
+              }
+              if (pos[s] < len[s]) best = min(best, U.raw[s][pos[s]]);
+            }
+            if (best == 0x7fffffff) break;
+            uint8_t mk = 0;
+            for (int s = 0; s < 2; ++s)
+              if (pos[s] < len[s] && U.raw[s][pos[s]] == best) {
+                mk |= (uint8_t)(1u << s);
+                prev[s] = best;
+                ++pos[s];
+                ++U.cnt[s];
+              }
+            U.ulist[nu] = best;
+            U.umask[nu] = mk;
+            ++nu;
+          }
+          U.nu = nu;
+          U.lin_empty[0] = U.cnt[0] >= p.nb;
+          U.lin_empty[1] = U.cnt[1] >= p.nb;
+          if (err) M.err = 1;
+          mbar_arrive(&M.list_full[buf]);
+          // K and V of every union entry, gathered by block index; the Q
+          // tiles go out after the first entry so that its K/V load overlaps
+          // the previous unit's tail.
+          auto load_kv = [&](int j) -> bool {
+            const int blk = U.ulist[j];
+            for (int kv = 0; kv < 2; ++kv) {
+              const int slot = g % NR;
+              if (g >= (uint32_t)NR && !mbar_wait(&M.ring_empty[slot], ((g / NR) - 1) & 1, abort)) return false;
+              mbar_expect_tx(&M.ring_full[slot], TILE);
+              const CUtensorMap* mp = kv ? &tmV : &tmK;
+              for (int ka = 0; ka < 2; ++ka)
+                tma_load_4d(smem + Ly::ring_off + slot * TILE + ka * (BN * 128), mp, &M.ring_full[slot],
+                            ka * 64, h, blk * BN, b);
+              ring_par[slot] = (g / NR) & 1;
+              ++g;
+            }
+            return true;
+          };
+          if (nu > 0) ok = load_kv(0);
+          for (int s = 0; s < 2 && ok; ++s) {
+            if (!U.active[s]) continue;
+            if (uc[s] >= 1 && !(ok = mbar_wait(&M.q_empty[s], (uc[s] - 1) & 1, abort))) break;
+            mbar_expect_tx(&M.q_full[s], TILE);
+            for (int ka = 0; ka < 2; ++ka)
+              tma_load_4d(smem + Ly::q_off + s * TILE + ka * (BM * 128), &tmQ, &M.q_full[s], ka * 64, h,
+                          U.a[s] * BM, b);
+            q_par[s] = uc[s] & 1;
+            ++uc[s];
+          }
+          for (int j = 1; ok && j < nu; ++j) ok = load_kv(j);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        __syncwarp();
+      }
+      // Drain: copies complete on their own; wait (bounded) for the last ones.
+      if (lane == 0) {
+        int no_abort = 0;
+        for (int i = 0; i < NR; ++i)
+          if (ring_par[i] >= 0) mbar_wait(&M.ring_full[i], ring_par[i], &no_abort);
+        for (int i = 0; i < 2; ++i)
+          if (q_par[i] >= 0) mbar_wait(&M.q_full[i], q_par[i], &no_abort);
+        if (no_abort) *abort = 1;
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ================================================================ MMA issuer
+      constexpr uint32_t idesc_s = instr_desc(kFmtBF16, kFmtBF16, false, false, 128, BN);
+      constexpr uint32_t idesc_pv = instr_desc(kFmtBF16, kFmtBF16, false, true, 128, D);
+      constexpr uint32_t idesc_qt = instr_desc(kFmtBF16, kFmtBF16, false, false, 128, R);
+      constexpr uint32_t idesc_l = instr_desc(kFmtBF16, kFmtBF16, false, true, 128, D);
+      const uint32_t sQ = smem_u32(smem + Ly::q_off);
+      const uint32_t sR = smem_u32(smem + Ly::ring_off);
+      const uint32_t sPT = smem_u32(smem + Ly::pt_off);
+      const uint32_t sAcc = smem_u32(smem + Ly::acc_off);
+      // k-step-0 descriptors of the Q tiles, of the ring slots as K
+      // (K-major) and as V (MN-major), all with 128-byte swizzle
+      // (a tile further on is TILE / 16 more in the start-address field)
+      const uint64_t dq0[2] = {desc_k_sw128(sQ, BM, 0), desc_k_sw128(sQ + TILE, BM, 0)};
+      const uint64_t dr_base = desc_k_sw128(sR, BN, 0);
+      const uint64_t dv_base = smem_desc(sR, BN * 128, 1024, kSwizzle128B);
+      uint32_t g = 0, np[2] = {0, 0}, uc[2] = {0, 0};
+      int users[NR];
+      for (int i = 0; i < NR; ++i) users[i] = 0;
+      bool ok = true;
+      for (int u = 0; ok && u < my_units; ++u) {
+        const int buf = u & 1;
+        if (!(ok = mbar_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+        const UnitList& U = M.L[buf];
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (ok && U.active[s]) ok = mbar_wait(&M.q_full[s], uc[s] & 1, abort);
+        if (!ok) break;
+        int pend_v[2] = {-1, -1};  // ring index of the V tile a slot's next P.V uses
+        bool first_pv[2] = {true, true};
+        auto issue_pv = [&](int s) -> bool {
+          if (!mbar_wait(&M.p_full[s], np[s] & 1, abort)) return false;
+          // the previous unit's epilogue must have read O first
+          if (first_pv[s] && uc[s] >= 1 && !mbar_wait(&M.o_free[s], (uc[s] - 1) & 1, abort)) return false;
+          ++np[s];
+          const uint32_t gv = (uint32_t)pend_v[s];
+          if (!mbar_wait(&M.ring_full[gv % NR], (gv / NR) & 1, abort)) return false;
+          tc_fence_after();
+          const uint64_t dv = dv_base + (uint64_t)(gv % NR) * (TILE >> 4);
+          const uint32_t acc0 = first_pv[s] ? 0u : 1u;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tm + o_col(s), tm + s_col(s) + Ly::P_OFF + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4),
+                   idesc_pv, kk == 0 ? acc0 : 1u);
+          first_pv[s] = false;
+          if (--users[gv % NR] == 0) mma_commit(&M.ring_empty[gv % NR]);
+          pend_v[s] = -1;
+          return true;
+        };
+        for (int j = 0; ok && j < U.nu; ++j) {
+          const uint32_t gk = g, gv = g + 1;
+          g += 2;
+          if (!(ok = mbar_wait(&M.ring_full[gk % NR], (gk / NR) & 1, abort))) break;
+          const int mk = U.umask[j];
+          users[gv % NR] = __popc(mk);
+          // Every pending P.V goes out now, also for a slot that skips this
+          // block: a deferred P.V would pin its V tile in the ring.
+#pragma unroll
+          for (int s = 0; s < 2; ++s) {
+            if (ok && pend_v[s] >= 0) ok = issue_pv(s);
+            if (!ok || !((mk >> s) & 1)) continue;
+            tc_fence_after();
+            const uint64_t dq = dq0[s], dk = dr_base + (uint64_t)(gk % NR) * (TILE >> 4);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_ss(tm + s_col(s), dq + kstep_k_sw128(BM, kk), dk + kstep_k_sw128(BN, kk), idesc_s,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(&M.s_full[s]);
+            pend_v[s] = (int)gv;
+          }
+          if (ok) mma_commit(&M.ring_empty[gk % NR]);
+        }
+#pragma unroll
+        for (int s = 0; s < 2; ++s)
+          if (ok && pend_v[s] >= 0) ok = issue_pv(s);
+        if (!ok) break;
+        // tile end: q P_h into the (now free) S columns; Q is then free for
+        // the next unit.  Then O += rho'_q S_U with rho'_q read from tensor
+        // memory (written by the softmax warps) and S_U from the gather.
+        if (!(ok = mbar_wait(&M.pt_full, u & 1, abort))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (!U.active[s]) continue;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tm + s_col(s), dq0[s] + kstep_k_sw128(BM, kk), desc_k_sw128(sPT, 32, kk), idesc_qt,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(&M.qt_full[s]);
+          mma_commit(&M.q_empty[s]);
+        }
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          if (!ok || !U.active[s]) continue;
+          if (!(ok = mbar_wait(&M.lin_ready[s], uc[s] & 1, abort))) continue;
+          if (!(ok = mbar_wait(&M.zu_ready[s], uc[s] & 1, abort))) continue;
+          tc_fence_after();
+          const uint32_t suh = sAcc + s * (R * D * 4), sul = suh + Ly::SU_BYTES;
+          const uint32_t a_hi = tm + s_col(s) + 32, a_lo = a_hi + R / 2;
+#pragma unroll
+          for (int kk = 0; kk < R / 16; ++kk) {
+            const uint64_t bh_ = smem_desc(suh + kk * 2048, R * 128, 1024, kSwizzle128B);
+            const uint64_t bl_ = smem_desc(sul + kk * 2048, R * 128, 1024, kSwizzle128B);
+            // a slot without any kept block has no P.V in O yet
+            mma_ts(tm + o_col(s), a_hi + kk * 8, bh_, idesc_l, (kk == 0 && U.cnt[s] == 0) ? 0u : 1u);
+            mma_ts(tm + o_col(s), a_hi + kk * 8, bl_, idesc_l, 1u);
+            mma_ts(tm + o_col(s), a_lo + kk * 8, bh_, idesc_l, 1u);
+          }
+          mma_commit(&M.l_done[s]);
+          ++uc[s];
+        }
+        if (!ok) break;
+        mbar_arrive(&M.list_empty[buf]);
+      }
+      mma_commit(&M.mma_final);
+      int no_abort = 0;
+      mbar_wait(&M.mma_final, 0, &no_abort);
+      if (no_abort) *abort = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+  if (tid == 0 && p.dev_err && (M.abort || M.err))
+    atomicOr(p.dev_err, (M.abort ? ROLA_DEVERR_TIMEOUT : 0) | (M.err ? ROLA_DEVERR_BAD_INDEX : 0));
+}
+
+static bool make_map(CUtensorMap* m, const void* base, const rola_shape_t* s) {
+  auto enc = rola_host::encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)s->d, (cuuint64_t)s->H, (cuuint64_t)s->N, (cuuint64_t)s->B};
+  const cuuint64_t strides[3] = {(cuuint64_t)s->d * 2, (cuuint64_t)s->H * s->d * 2,
+                                 (cuuint64_t)s->N * s->H * s->d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+template <int R>
+static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            Params prm, cudaStream_t cs) {
+  using Ly = Layout<R>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, s) || !make_map(&mk, k, s) || !make_map(&mv, v, s)) return ROLA_ERR_CUDA;
+  const size_t smem = Ly::misc_off + sizeof(Misc) + 1024;
+  auto kern = rola_attn_pair_kernel<R>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  const int grid = prm.units < sm_count() ? prm.units : sm_count();
+  kern<<<grid, kThreads, smem, cs>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+}
+
+}  // namespace pairk
+
+// Used by rola_attention_fwd for d = 128, 128-token blocks, k_b <= 256 and a
+// latent grid whose rotary table fits in shared memory.
+bool pair_kernel_supports(const rola_shape_t* s) {
+  if (!(s->d == 128 && s->block == 128 && s->k_b <= pairk::kMaxKept && (s->r == 16 || s->r == 32)))
+    return false;
+  const int rh = 2 * (s->r / 6), rt = s->r - 2 * rh;
+  const long long entries = (long long)s->T * (rt / 2) + (long long)(s->Hg + s->W) * (rh / 2);
+  return entries <= pairk::kTabCap;
+}
+
+rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const int32_t* idx, const uint16_t* P,
+                                 const float* S_blk, const float* z_blk, const float* S_glb,
+                                 const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
+                                 cudaStream_t cs) {
+  pairk::Params prm{};
+  prm.B = s->B;
+  prm.H = s->H;
+  prm.N = s->N;
+  prm.nb = rola_num_blocks(s);
+  prm.kb = s->k_b;
+  prm.T = s->T;
+  prm.Hg = s->Hg;
+  prm.W = s->W;
+  prm.npairs = (prm.nb + 1) / 2;
+  prm.units = s->B * s->H * prm.npairs;
+  prm.scale_log2 = (float)(1.4426950408889634 / sqrt((double)s->d));
+  prm.idx = idx;
+  prm.P = P;
+  prm.S_blk = S_blk;
+  prm.z_blk = z_blk;
+  prm.S_glb = S_glb;
+  prm.z_glb = z_glb;
+  prm.gate = gate;
+  prm.out = out;
+  prm.dev_err = dev_err;
+  rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
+  {
+    // rotary cos/sin table layout: per axis a block of len_a x npairs_a entries
+    const int npairs = s->r / 2;
+    const int len[3] = {s->T, s->Hg, s->W};
+    int np_axis[3] = {0, 0, 0};
+    for (int pr = 0; pr < npairs; ++pr) ++np_axis[prm.rope.axis[pr]];
+    const long long off[3] = {0, (long long)len[0] * np_axis[0],
+                              (long long)len[0] * np_axis[0] + (long long)len[1] * np_axis[1]};
+    const long long total = off[2] + (long long)len[2] * np_axis[2];
+    int first = 0, m_axis[3] = {0, 0, 0};
+    for (int pr = 0; pr < npairs; ++pr) {
+      const int ax = prm.rope.axis[pr];
+      prm.tab_base[pr] = (int)(off[ax] + m_axis[ax]++);
+      prm.tab_stride[pr] = np_axis[ax];
+      prm.tab_first[pr] = first;
+      first += len[ax];
+    }
+    prm.tab_first[npairs] = first;
+    prm.tab_entries = (int)total;
+  }
+  if (s->r == 32) return pairk::launch<32>(s, q, k, v, prm, cs);
+  return pairk::launch<16>(s, q, k, v, prm, cs);
+}
+
+}  // namespace rola

@@ -241,6 +241,48 @@ ROLA_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// The same 32-column load / store into elements [OFF, OFF + 32) of a larger
+// register array (constant indices keep the array in registers).
+template <int OFF, int N>
+ROLA_DEV void tmem_ld32_at(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(OFF + 32 <= N, "range");
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[OFF + 0]), "=r"(r[OFF + 1]), "=r"(r[OFF + 2]), "=r"(r[OFF + 3]), "=r"(r[OFF + 4]),
+        "=r"(r[OFF + 5]), "=r"(r[OFF + 6]), "=r"(r[OFF + 7]), "=r"(r[OFF + 8]), "=r"(r[OFF + 9]),
+        "=r"(r[OFF + 10]), "=r"(r[OFF + 11]), "=r"(r[OFF + 12]), "=r"(r[OFF + 13]),
+        "=r"(r[OFF + 14]), "=r"(r[OFF + 15]), "=r"(r[OFF + 16]), "=r"(r[OFF + 17]),
+        "=r"(r[OFF + 18]), "=r"(r[OFF + 19]), "=r"(r[OFF + 20]), "=r"(r[OFF + 21]),
+        "=r"(r[OFF + 22]), "=r"(r[OFF + 23]), "=r"(r[OFF + 24]), "=r"(r[OFF + 25]),
+        "=r"(r[OFF + 26]), "=r"(r[OFF + 27]), "=r"(r[OFF + 28]), "=r"(r[OFF + 29]),
+        "=r"(r[OFF + 30]), "=r"(r[OFF + 31])
+      : "r"(taddr));
+}
+template <int OFF, int N>
+ROLA_DEV void tmem_st32_at(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(OFF + 32 <= N, "range");
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31, %32};" ::"r"(taddr),
+      "r"(r[OFF + 0]), "r"(r[OFF + 1]), "r"(r[OFF + 2]), "r"(r[OFF + 3]), "r"(r[OFF + 4]),
+      "r"(r[OFF + 5]), "r"(r[OFF + 6]), "r"(r[OFF + 7]), "r"(r[OFF + 8]), "r"(r[OFF + 9]),
+      "r"(r[OFF + 10]), "r"(r[OFF + 11]), "r"(r[OFF + 12]), "r"(r[OFF + 13]), "r"(r[OFF + 14]),
+      "r"(r[OFF + 15]), "r"(r[OFF + 16]), "r"(r[OFF + 17]), "r"(r[OFF + 18]), "r"(r[OFF + 19]),
+      "r"(r[OFF + 20]), "r"(r[OFF + 21]), "r"(r[OFF + 22]), "r"(r[OFF + 23]), "r"(r[OFF + 24]),
+      "r"(r[OFF + 25]), "r"(r[OFF + 26]), "r"(r[OFF + 27]), "r"(r[OFF + 28]), "r"(r[OFF + 29]),
+      "r"(r[OFF + 30]), "r"(r[OFF + 31])
+      : "memory");
+}
+
+ROLA_DEV void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 ROLA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -271,6 +313,58 @@ ROLA_DEV void rope_sincos(int pos, double freq, float* s, float* c) {
 
 // phi(u) = elu(u) + 1.
 ROLA_DEV float phi(float u) { return u > 0.f ? u + 1.f : expf(u); }
+
+// ---------------------------------------------------------------- packed fp32
+
+ROLA_DEV uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+ROLA_DEV void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// (a * b + c) on two lanes at once
+ROLA_DEV uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+ROLA_DEV uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+ROLA_DEV float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^y for two lanes on the FMA pipe (offloads the special-function unit).
+// Range reduction: y = n + f with n = rint(y) taken from y + 1.5 * 2^23
+// (round to nearest) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
+// fitted here to 2^f in relative error on [-1/2, 1/2] (max relative error
+// 7.5e-5 in float32); 2^n applied by adding n to the exponent field.  y is
+// clamped below at -126 (results there are below 2^-125 and negligible).
+constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f,
+                kExp2C3 = 0.055171624f;
+ROLA_DEV void exp2_poly2(float y0, float y1, float& e0, float& e1) {
+  const uint64_t shift = f32x2(12582912.f, 12582912.f);
+  const uint64_t nshift = f32x2(-12582912.f, -12582912.f);
+  const uint64_t y = f32x2(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
+  const uint64_t t = fadd2(y, shift);           // low bits hold rint(y)
+  const uint64_t n = fadd2(t, nshift);          // rint(y) as float
+  const uint64_t fr = ffma2(n, f32x2(-1.f, -1.f), y);
+  uint64_t p = ffma2(fr, f32x2(kExp2C3, kExp2C3), f32x2(kExp2C2, kExp2C2));
+  p = ffma2(p, fr, f32x2(kExp2C1, kExp2C1));
+  p = ffma2(p, fr, f32x2(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f32x2_split(p, p0, p1);
+  f32x2_split(t, t0, t1);
+  e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
 
 // ---------------------------------------------------------------- misc
 
