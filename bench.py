@@ -204,65 +204,35 @@ def run_gpu(args) -> int:
     gate = torch.from_numpy(inp["gate"]).cuda()
     stream = torch.cuda.current_stream()
 
-    # persistent buffers for the three stages (the layer's own workspace layout)
-    nb = w.n_blocks
-    idx = torch.empty((w.B, w.H, nb, w.k_b), dtype=torch.int32, device="cuda")
-    S_blk = torch.empty((w.B, w.H, nb, w.r, w.d), dtype=torch.float32, device="cuda")
-    z_blk = torch.empty((w.B, w.H, nb, w.r), dtype=torch.float32, device="cuda")
-    S_glb = torch.empty((w.B, w.H, w.r, w.d), dtype=torch.float32, device="cuda")
-    z_glb = torch.empty((w.B, w.H, w.r), dtype=torch.float32, device="cuda")
+    # the layer's own entry point; three events split it into its two stages
+    layer = rb.Layer(shape)
     out = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device="cuda")
-    dev_err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    import ctypes
-    L = rb.lib()
-    cs = shape.c()
-    sel_ws_bytes = L.rola_select_workspace_bytes(ctypes.byref(cs))
-    sel_ws = torch.empty(sel_ws_bytes, dtype=torch.uint8, device="cuda")
-    sptr = ctypes.c_void_p(stream.cuda_stream)
-    P_ = lambda t: ctypes.c_void_p(t.data_ptr())
+    stage_names = ("select+states", "attention")
+    launches_per_step = rb.layer_launches(shape)
 
-    def select():
-        st = L.rola_select_blocks(ctypes.byref(cs), P_(q), P_(k), P_(idx), None, P_(sel_ws),
-                                  sel_ws_bytes, sptr)
-        assert st == 0, st
-
-    def states():
-        st = L.rola_block_states(ctypes.byref(cs), P_(k), P_(v), P_(P), P_(S_blk), P_(z_blk),
-                                 P_(S_glb), P_(z_glb), sptr)
-        assert st == 0, st
-
-    def attention():
-        st = L.rola_attention_fwd(ctypes.byref(cs), P_(q), P_(k), P_(v), P_(idx), P_(P), P_(S_blk),
-                                  P_(z_blk), P_(S_glb), P_(z_glb), P_(gate), P_(out), P_(dev_err), sptr)
-        assert st == 0, st
-
-    stages = [("select", select, 3), ("states", states, 2), ("attention", attention, 1)]
     for _ in range(args.warmup):
-        for _, fn, _ in stages:
-            fn()
+        layer(q, k, v, P, gate, out=out, stream=stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         for s in range(K):
-            ev[s][0].record(stream)
-            for i, (_, fn, _) in enumerate(stages):
-                fn()
-                ev[s][i + 1].record(stream)
+            layer(q, k, v, P, gate, out=out, stream=stream, events=ev[s])
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    assert int(dev_err.item()) == 0, f"device error flag {int(dev_err.item())}"
+    err = int(layer.dev_err.item())
+    assert err == 0, f"device error flag {err}"
 
     per_stage = {nm: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)]
-                 for i, (nm, _, _) in enumerate(stages)}
-    total_ms = ev[0][0].elapsed_time(ev[K - 1][len(stages)])
+                 for i, nm in enumerate(stage_names)}
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
     t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -315,12 +285,12 @@ def run_gpu(args) -> int:
             "kernels_ms": {nm: statistics.mean(x) for nm, x in per_stage.items()},
             "attention_tflops": achieved,
             "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
-            "roofline": {"bound": "tensor", "kernel": "rola_attn_kernel", "achieved": achieved,
+            "roofline": {"bound": "tensor", "kernel": "rola_attn_pair_kernel", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                          "peak_source": peaks["source"] + " bf16 burst"},
             "e2e": e2e,
-            "gpu_launches": K * sum(n for _, _, n in stages),
+            "gpu_launches": K * launches_per_step,
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline:
@@ -335,7 +305,7 @@ def run_gpu(args) -> int:
 def kernel_hash() -> str:
     import hashlib
     h = hashlib.sha1()
-    for nm in ("rola_attention.cu", "rola_common.cuh"):
+    for nm in ("rola_attention.cu", "rola_attention_pair.cu", "rola_common.cuh"):
         with open(os.path.join(ROOT, "sparse_linear_attention_mean_b200", "csrc", nm), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]

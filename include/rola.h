@@ -164,6 +164,20 @@ rola_status_t rola_layer_fwd(const rola_shape_t* shape, const uint16_t* q, const
                              int32_t* idx_out, void* ws, size_t ws_bytes, int32_t* dev_err,
                              void* stream);
 
+/* rola_layer_fwd with CUDA events recorded on `stream` at its stage
+ * boundaries, for profiling: events[0] before the first kernel, events[1]
+ * once the selection and the block states are done, events[2] after the
+ * attention kernel.  `events` points to three cudaEvent_t the caller created
+ * (or is NULL, which makes the call identical to rola_layer_fwd). */
+rola_status_t rola_layer_fwd_timed(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
+                                   const uint16_t* v, const uint16_t* P, const float* gate,
+                                   uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
+                                   int32_t* dev_err, void* stream, void* const* events);
+
+/* Number of kernels one rola_layer_fwd call launches for `shape` (0 for an
+ * invalid or unsupported shape); memory copies are not counted. */
+int rola_layer_kernel_launches(const rola_shape_t* shape);
+
 /* Device staging the host-buffer variant needs on top of the layer
  * workspace: q, k, v, P, gate and out. */
 size_t rola_layer_host_workspace_bytes(const rola_shape_t* shape);

@@ -23,7 +23,8 @@ DEVERR_TIMEOUT = 0x2
 EXPORTS = [
     "rola_status_string", "rola_num_blocks", "rola_kb_from_sparsity",
     "rola_select_workspace_bytes", "rola_select_blocks", "rola_block_states",
-    "rola_attention_fwd", "rola_layer_workspace_bytes", "rola_layer_fwd",
+    "rola_attention_fwd", "rola_layer_workspace_bytes", "rola_layer_fwd", "rola_layer_fwd_timed",
+    "rola_layer_kernel_launches",
     "rola_layer_host_workspace_bytes", "rola_layer_fwd_host",
     "fp8_quantize_rows_bf16", "fp8_quantize_weight", "fp8_gemm_w8a8",
     "fp8_linear_workspace_bytes", "fp8_linear_w8a8",
@@ -100,6 +101,11 @@ def lib() -> ctypes.CDLL:
         L.rola_attention_fwd.argtypes = [sp] + [vp] * 12 + [vp]
         L.rola_layer_fwd.restype = ctypes.c_int
         L.rola_layer_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+        L.rola_layer_fwd_timed.restype = ctypes.c_int
+        L.rola_layer_fwd_timed.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp,
+                                           ctypes.POINTER(ctypes.c_void_p)]
+        L.rola_layer_kernel_launches.restype = ctypes.c_int
+        L.rola_layer_kernel_launches.argtypes = [sp]
         L.rola_layer_fwd_host.restype = ctypes.c_int
         L.rola_layer_fwd_host.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         L.fp8_quantize_rows_bf16.restype = ctypes.c_int
@@ -231,7 +237,9 @@ class Layer:
         self.ws = _ws(self.ws_bytes, device)
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
 
-    def __call__(self, q, k, v, P, gate, *, out=None, idx_out=None, stream=None):
+    def __call__(self, q, k, v, P, gate, *, out=None, idx_out=None, stream=None, events=None):
+        """events: optional three torch.cuda.Event(enable_timing=True), recorded
+        before the layer, after selection + states, and after the attention."""
         s = self.shape
         act = (s.B, s.N, s.H, s.d)
         for t, nm in ((q, "q"), (k, "k"), (v, "v")):
@@ -242,11 +250,32 @@ class Layer:
             out = torch.empty(act, dtype=torch.bfloat16, device=q.device)
         if idx_out is not None:
             _need(idx_out, torch.int32, (s.B, s.H, s.n_blocks, s.k_b), "idx_out")
-        _check(lib().rola_layer_fwd(ctypes.byref(self.c), _ptr(q), _ptr(k), _ptr(v), _ptr(P),
-                                    _ptr(gate), _ptr(out), _ptr(idx_out), _ptr(self.ws),
-                                    self.ws_bytes, _ptr(self.dev_err), _stream(stream)),
-               "rola_layer_fwd")
+        if events is None:
+            _check(lib().rola_layer_fwd(ctypes.byref(self.c), _ptr(q), _ptr(k), _ptr(v), _ptr(P),
+                                        _ptr(gate), _ptr(out), _ptr(idx_out), _ptr(self.ws),
+                                        self.ws_bytes, _ptr(self.dev_err), _stream(stream)),
+                   "rola_layer_fwd")
+        else:
+            if len(events) != 3:
+                raise ValueError("events: three torch.cuda.Event")
+            for e in events:
+                if not e.cuda_event:  # torch creates the handle on first record
+                    e.record(stream if stream is not None else torch.cuda.current_stream())
+            ev = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
+            _check(lib().rola_layer_fwd_timed(ctypes.byref(self.c), _ptr(q), _ptr(k), _ptr(v), _ptr(P),
+                                              _ptr(gate), _ptr(out), _ptr(idx_out), _ptr(self.ws),
+                                              self.ws_bytes, _ptr(self.dev_err), _stream(stream), ev),
+                   "rola_layer_fwd_timed")
         return out
+
+
+def layer_launches(shape: Shape) -> int:
+    """Kernels one layer call launches for `shape`."""
+    c = shape.c()
+    n = lib().rola_layer_kernel_launches(ctypes.byref(c))
+    if n <= 0:
+        raise RolaError("invalid or unsupported shape")
+    return n
 
 
 class HostLayer:

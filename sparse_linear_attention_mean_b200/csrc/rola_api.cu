@@ -81,9 +81,49 @@ int rope_frequencies(int r, float base, double* freq, int* axis) {
   return p;
 }
 
+void rope_table_layout(const rola_shape_t* s, const int* axis, RopeTabLayout* out) {
+  const int npairs = s->r / 2;
+  const int len[3] = {s->T, s->Hg, s->W};
+  int np_axis[3] = {0, 0, 0};
+  for (int pr = 0; pr < npairs; ++pr) ++np_axis[axis[pr]];
+  const long long off[3] = {0, (long long)len[0] * np_axis[0],
+                            (long long)len[0] * np_axis[0] + (long long)len[1] * np_axis[1]};
+  int first = 0, m_axis[3] = {0, 0, 0};
+  for (int pr = 0; pr < npairs; ++pr) {
+    const int ax = axis[pr];
+    out->base[pr] = (int)(off[ax] + m_axis[ax]++);
+    out->stride[pr] = np_axis[ax];
+    out->first[pr] = first;
+    first += len[ax];
+  }
+  out->first[npairs] = first;
+  out->entries = (int)(off[2] + (long long)len[2] * np_axis[2]);
+}
+
+bool make_act_map(CUtensorMap* m, const void* base, const rola_shape_t* s, int box_rows) {
+  auto enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)s->d, (cuuint64_t)s->H, (cuuint64_t)s->N, (cuuint64_t)s->B};
+  const cuuint64_t strides[3] = {(cuuint64_t)s->d * 2, (cuuint64_t)s->H * s->d * 2,
+                                 (cuuint64_t)s->N * s->H * s->d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
 }  // namespace rola_host
 
 using rola_internal::check_shape;
+using rola_internal::round_up;
 
 extern "C" const char* rola_status_string(rola_status_t s) {
   switch (s) {
@@ -113,10 +153,29 @@ extern "C" size_t rola_layer_workspace_bytes(const rola_shape_t* s) {
   return rola_internal::layer_ws(s).total;
 }
 
+extern "C" int rola_layer_kernel_launches(const rola_shape_t* s) {
+  if (check_shape(s) != ROLA_OK) return 0;
+  // fused path: prep, score, top-k, state totals, attention;
+  // otherwise: pool, score, top-k, block states, state totals, attention
+  return rola::prep_kernel_supports(s) ? 5 : 6;
+}
+
 extern "C" rola_status_t rola_layer_fwd(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
                                         const uint16_t* v, const uint16_t* P, const float* gate,
                                         uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
                                         int32_t* dev_err, void* stream) {
+  return rola_layer_fwd_timed(s, q, k, v, P, gate, out, idx_out, ws, ws_bytes, dev_err, stream, nullptr);
+}
+
+extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint16_t* q,
+                                              const uint16_t* k, const uint16_t* v, const uint16_t* P,
+                                              const float* gate, uint16_t* out, int32_t* idx_out,
+                                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream,
+                                              void* const* events) {
+  auto mark = [&](int i) -> bool {
+    return !events || cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]),
+                                      reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess;
+  };
   rola_status_t st = check_shape(s);
   if (st != ROLA_OK) return st;
   const rola_internal::LayerWs L = rola_internal::layer_ws(s);
@@ -127,13 +186,36 @@ extern "C" rola_status_t rola_layer_fwd(const rola_shape_t* s, const uint16_t* q
   float* z_blk = reinterpret_cast<float*>(base + L.z_blk);
   float* S_glb = reinterpret_cast<float*>(base + L.S_glb);
   float* z_glb = reinterpret_cast<float*>(base + L.z_glb);
-  st = rola_select_blocks(s, q, k, idx, nullptr, base + L.select, L.idx - L.select, stream);
-  if (st != ROLA_OK) return st;
-  st = rola_block_states(s, k, v, P, S_blk, z_blk, S_glb, z_glb, stream);
-  if (st != ROLA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (!mark(0)) return ROLA_ERR_CUDA;
+  if (rola::prep_kernel_supports(s)) {
+    // one pass over q, k, v: block means for the selector and block states
+    if (!q || !k || !v || !P || !gate || !out) return ROLA_ERR_INVALID_ARG;
+    if (!rola_host::aligned(q, 16) || !rola_host::aligned(k, 16) || !rola_host::aligned(v, 16) ||
+        !rola_host::aligned(P, 16))
+      return ROLA_ERR_ALIGNMENT;
+    if (rola_num_blocks(s) > 1024) return ROLA_ERR_UNSUPPORTED;
+    const size_t pooled = (size_t)s->B * s->H * rola_num_blocks(s) * s->d;
+    double* qbar = reinterpret_cast<double*>(base + L.select);
+    double* kbar = qbar + pooled;
+    double* sigma = reinterpret_cast<double*>(base + L.select + round_up(2 * pooled * sizeof(double), 256));
+    st = rola::launch_prep_kernel(s, q, k, v, P, qbar, kbar, S_blk, z_blk, dev_err, cs);
+    if (st != ROLA_OK) return st;
+    st = rola::select_from_pooled(s, qbar, kbar, sigma, idx, cs);
+    if (st != ROLA_OK) return st;
+    st = rola::launch_states_total(s, S_blk, z_blk, S_glb, z_glb, cs);
+    if (st != ROLA_OK) return st;
+  } else {
+    st = rola_select_blocks(s, q, k, idx, nullptr, base + L.select, L.idx - L.select, stream);
+    if (st != ROLA_OK) return st;
+    st = rola_block_states(s, k, v, P, S_blk, z_blk, S_glb, z_glb, stream);
+    if (st != ROLA_OK) return st;
+  }
+  if (!mark(1)) return ROLA_ERR_CUDA;
   st = rola_attention_fwd(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
                           stream);
   if (st != ROLA_OK) return st;
+  if (!mark(2)) return ROLA_ERR_CUDA;
   if (idx_out) {
     const size_t bytes = (size_t)s->B * s->H * rola_num_blocks(s) * s->k_b * sizeof(int32_t);
     if (cudaMemcpyAsync(idx_out, idx, bytes, cudaMemcpyDeviceToDevice,

@@ -727,37 +727,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicOr(p.dev_err, (M.abort ? ROLA_DEVERR_TIMEOUT : 0) | (M.err ? ROLA_DEVERR_BAD_INDEX : 0));
 }
 
-static bool make_map(CUtensorMap* m, const void* base, const rola_shape_t* s) {
-  auto enc = rola_host::encode_tiled_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)s->d, (cuuint64_t)s->H, (cuuint64_t)s->N, (cuuint64_t)s->B};
-  const cuuint64_t strides[3] = {(cuuint64_t)s->d * 2, (cuuint64_t)s->H * s->d * 2,
-                                 (cuuint64_t)s->N * s->H * s->d * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-static int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-  return n;
-}
-
 template <int R>
 static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                             Params prm, cudaStream_t cs) {
   using Ly = Layout<R>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, s) || !make_map(&mk, k, s) || !make_map(&mv, v, s)) return ROLA_ERR_CUDA;
+  if (!rola_host::make_act_map(&mq, q, s, 128) || !rola_host::make_act_map(&mk, k, s, 128) ||
+      !rola_host::make_act_map(&mv, v, s, 128))
+    return ROLA_ERR_CUDA;
   const size_t smem = Ly::misc_off + sizeof(Misc) + 1024;
   auto kern = rola_attn_pair_kernel<R>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ROLA_ERR_CUDA;
-  const int grid = prm.units < sm_count() ? prm.units : sm_count();
+  const int nsm = rola_host::sm_count();
+  const int grid = prm.units < nsm ? prm.units : nsm;
   kern<<<grid, kThreads, smem, cs>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
@@ -802,24 +785,14 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
   prm.dev_err = dev_err;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
   {
-    // rotary cos/sin table layout: per axis a block of len_a x npairs_a entries
-    const int npairs = s->r / 2;
-    const int len[3] = {s->T, s->Hg, s->W};
-    int np_axis[3] = {0, 0, 0};
-    for (int pr = 0; pr < npairs; ++pr) ++np_axis[prm.rope.axis[pr]];
-    const long long off[3] = {0, (long long)len[0] * np_axis[0],
-                              (long long)len[0] * np_axis[0] + (long long)len[1] * np_axis[1]};
-    const long long total = off[2] + (long long)len[2] * np_axis[2];
-    int first = 0, m_axis[3] = {0, 0, 0};
-    for (int pr = 0; pr < npairs; ++pr) {
-      const int ax = prm.rope.axis[pr];
-      prm.tab_base[pr] = (int)(off[ax] + m_axis[ax]++);
-      prm.tab_stride[pr] = np_axis[ax];
-      prm.tab_first[pr] = first;
-      first += len[ax];
+    rola_host::RopeTabLayout tl;
+    rola_host::rope_table_layout(s, prm.rope.axis, &tl);
+    for (int i = 0; i < 16; ++i) {
+      prm.tab_base[i] = tl.base[i];
+      prm.tab_stride[i] = tl.stride[i];
     }
-    prm.tab_first[npairs] = first;
-    prm.tab_entries = (int)total;
+    for (int i = 0; i < 17; ++i) prm.tab_first[i] = tl.first[i];
+    prm.tab_entries = tl.entries;
   }
   if (s->r == 32) return pairk::launch<32>(s, q, k, v, prm, cs);
   return pairk::launch<16>(s, q, k, v, prm, cs);

@@ -393,4 +393,20 @@ EncodeTiledFn encode_tiled_fn();
 // float64 (computed on the host once per launch; at most 64 pairs).
 int rope_frequencies(int r, float base, double* freq /* [r/2] */, int* axis /* [r/2] */);
 
+// Layout of a per-CTA cos/sin table of the rotary angles: pair pr at grid
+// position pos is entry base[pr] + pos * stride[pr]; pair pr fills entries
+// [first[pr], first[pr + 1]) in fill order; `entries` in total.
+struct RopeTabLayout {
+  int base[16], stride[16], first[17];
+  int entries;
+};
+void rope_table_layout(const rola_shape_t* s, const int* axis, RopeTabLayout* out);
+
+// 4-D TMA map over a [B, N, H, d] bf16 activation: box of 64 channels x 1
+// head x `box_rows` tokens, 128-byte swizzle, zero fill past N.
+bool make_act_map(CUtensorMap* m, const void* base, const rola_shape_t* s, int box_rows);
+
+// Streaming multiprocessors of the current device.
+int sm_count();
+
 }  // namespace rola_host

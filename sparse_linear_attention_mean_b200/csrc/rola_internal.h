@@ -21,3 +21,18 @@ struct LayerWs {
 LayerWs layer_ws(const rola_shape_t* s);
 
 }  // namespace rola_internal
+
+#ifdef __CUDACC__
+#include <cuda_runtime.h>
+namespace rola {
+// Internal launchers shared by the entry points.
+rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, const double* kbar,
+                                 double* sigma, int32_t* idx, cudaStream_t cs);
+bool prep_kernel_supports(const rola_shape_t* s);
+rola_status_t launch_prep_kernel(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint16_t* P, double* qbar, double* kbar,
+                                 float* S_blk, float* z_blk, int32_t* dev_err, cudaStream_t cs);
+rola_status_t launch_states_total(const rola_shape_t* s, const float* S_blk, const float* z_blk,
+                                  float* S_glb, float* z_glb, cudaStream_t cs);
+}  // namespace rola
+#endif

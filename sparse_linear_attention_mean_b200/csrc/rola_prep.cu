@@ -1,0 +1,370 @@
+// One pass over q, k and v for d = 128 and 128-token blocks: the float64
+// block means of q and k that the selector scores, and the linear-branch
+// states of every block, read from HBM once.
+//
+// SparkDiffusion write-up (0539edu.com news page), section 05: the sparse
+// branch keeps the important query-key blocks (selected here from block
+// means), and a rotary low-rank linear branch restores the dropped context
+// (per-block states S_j = rho^T V, z_j = sum psi, rho = R(t, y, x) phi(K P_h)).
+//
+// Persistent CTAs (256 threads) walk (batch, head, block) items.  Thread 0
+// TMA-loads the q, k and v tiles of the next item (128-byte swizzle) while
+// all warps work on the current one:
+//   * block sums of q and k over the valid tokens in float64 (exact for bf16),
+//     divided by the count;
+//   * K P_h with mma.sync, psi = phi(.), rho = rotation by a per-CTA cos/sin
+//     table of the 3-D rotary angles, written as bf16 hi + lo over the (then
+//     dead) q tile;
+//   * S_j^T = V^T rho with mma.sync (hi and lo parts), z_j = sum of psi.
+// The kernel is bound by HBM: 96 KB read and ~18 KB written per item.
+#include <math.h>
+
+#include "rola_common.cuh"
+#include "rola_internal.h"
+
+namespace rola {
+namespace prep {
+
+constexpr int kThreads = 256;
+constexpr int D = 128, BS = 128;
+constexpr uint32_t TILE = BS * D * 2;  // 32 KB
+constexpr int kTabCap = 1024;
+
+template <int R>
+struct Layout {
+  static constexpr uint32_t stage_bytes = 3 * TILE;  // q, k, v
+  static constexpr uint32_t pt_off = 2 * stage_bytes;
+  static constexpr int PS = R + 8;                   // padded row of P_h and rho (bf16)
+  static constexpr uint32_t misc_off = pt_off + D * PS * 2;
+  static constexpr uint32_t RHO_BYTES = BS * PS * 2;  // one of hi / lo, inside the q tile
+  static_assert(2 * RHO_BYTES <= TILE, "rho must fit in the q tile");
+};
+
+struct Misc {
+  uint64_t full[2];
+  int abort;
+  int cur_h;
+  float zpart[8][32];
+  float2 tab[kTabCap];
+};
+
+struct Params {
+  int B, H, N, nb, Hg, W, items;
+  int do_pool;
+  double* qbar;  // [B, H, nb, d] float64, or null
+  double* kbar;
+  const uint16_t* P;
+  float* S_blk;
+  float* z_blk;
+  int32_t* dev_err;
+  RopeTable rope;
+  int tab_base[16], tab_stride[16], tab_first[17];
+  int tab_entries;  // 0: table too large, sin/cos computed directly
+};
+
+ROLA_DEV void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+ROLA_DEV void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+ROLA_DEV void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Byte offset of element (row, col) of a [128 x 128] bf16 tile stored as two
+// 64-column atoms with the TMA 128-byte swizzle.
+ROLA_DEV uint32_t sw_off(int row, int col) {
+  return (uint32_t)((col >> 6) * (BS * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                    (col & 7) * 2);
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    rola_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using Ly = Layout<R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& M = *reinterpret_cast<Misc*>(smem + Ly::misc_off);
+  uint16_t* sP = reinterpret_cast<uint16_t*>(smem + Ly::pt_off);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int my_items =
+      p.items > (int)blockIdx.x ? (p.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (tid == 0) {
+    mbar_init(&M.full[0], 1);
+    mbar_init(&M.full[1], 1);
+    M.abort = 0;
+    M.cur_h = -1;
+    fence_barrier_init();
+  }
+  for (int e = tid; e < p.tab_entries; e += kThreads) {
+    int pr = 0;
+    while (pr + 1 < R / 2 && e >= p.tab_first[pr + 1]) ++pr;
+    const int pos = e - p.tab_first[pr];
+    float sn, cs;
+    rope_sincos(pos, p.rope.freq[pr], &sn, &cs);
+    M.tab[p.tab_base[pr] + pos * p.tab_stride[pr]] = make_float2(cs, sn);
+  }
+  __syncthreads();
+  volatile int* abort = &M.abort;
+
+  auto decode = [&](int it, int& b, int& h, int& blk) {
+    const int id = (int)blockIdx.x + it * (int)gridDim.x;
+    blk = id % p.nb;
+    h = (id / p.nb) % p.H;
+    b = id / (p.nb * p.H);
+  };
+  auto issue = [&](int it) {
+    int b, h, blk;
+    decode(it, b, h, blk);
+    const int st = it & 1;
+    uint8_t* base = smem + st * Ly::stage_bytes;
+    mbar_expect_tx(&M.full[st], p.do_pool ? 3 * TILE : 2 * TILE);
+    for (int ka = 0; ka < 2; ++ka) {
+      if (p.do_pool) tma_load_4d(base + ka * (BS * 128), &tmQ, &M.full[st], ka * 64, h, blk * BS, b);
+      tma_load_4d(base + TILE + ka * (BS * 128), &tmK, &M.full[st], ka * 64, h, blk * BS, b);
+      tma_load_4d(base + 2 * TILE + ka * (BS * 128), &tmV, &M.full[st], ka * 64, h, blk * BS, b);
+    }
+  };
+  if (tid == 0 && my_items > 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    issue(0);
+  }
+
+  bool ok = true;
+  int it = 0;
+  for (; ok && it < my_items; ++it) {
+    const int st = it & 1;
+    // the other stage was released by the __syncthreads closing the last item
+    if (tid == 0 && it + 1 < my_items) issue(it + 1);
+    int b, h, blk;
+    decode(it, b, h, blk);
+    const size_t bh = (size_t)b * p.H + h;
+    const int tok0 = blk * BS;
+    const int valid = min(BS, p.N - tok0);
+    uint8_t* sq = smem + st * Ly::stage_bytes;
+    uint8_t* sk = sq + TILE;
+    uint8_t* sv = sk + TILE;
+    // P_h (rows d, padded) when the head changes
+    if (h != M.cur_h) {
+      for (int e = tid; e < D * (R / 8); e += kThreads) {
+        const int row = e / (R / 8), ch = e % (R / 8);
+        *reinterpret_cast<uint4*>(sP + row * Ly::PS + ch * 8) =
+            *reinterpret_cast<const uint4*>(p.P + ((size_t)h * D + row) * R + ch * 8);
+      }
+      __syncthreads();
+      if (tid == 0) M.cur_h = h;
+    }
+    if (!(ok = mbar_wait(&M.full[st], (it >> 1) & 1, abort))) break;
+
+    // ---- block means of q and k (float64: the bf16 sums are exact)
+    if (p.do_pool) {
+      const uint8_t* tile = tid < 128 ? sq : sk;
+      const int c = tid & 127;
+      double acc = 0.0;
+      for (int r = 0; r < valid; ++r)
+        acc += (double)bf16_lo(*reinterpret_cast<const uint16_t*>(tile + sw_off(r, c)));
+      double* dst = tid < 128 ? p.qbar : p.kbar;
+      dst[(bh * p.nb + blk) * D + c] = acc / (double)valid;
+    }
+
+    // ---- kt = K P_h : warp w owns token rows [16w, 16w + 16)
+    constexpr int NT = R / 8;
+    float acc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+    {
+      const uint32_t kbase = smem_u32(sk), pbase = smem_u32(sP);
+      const int arow = warp * 16 + (lane & 15);
+#pragma unroll
+      for (int kk = 0; kk < D; kk += 16) {
+        uint32_t a[4];
+        ldsm_x4(a, kbase + sw_off(arow, kk + (lane >> 4) * 8));
+#pragma unroll
+        for (int nj = 0; nj < NT; nj += 2) {
+          uint32_t bb[4];
+          ldsm_x4_t(bb, pbase + ((kk + (lane & 15)) * Ly::PS + nj * 8 + (lane >> 4) * 8) * 2);
+          mma16816(acc[nj], a, bb[0], bb[1]);
+          mma16816(acc[nj + 1], a, bb[2], bb[3]);
+        }
+      }
+    }
+    __syncthreads();  // everyone is done with the q tile (pooling): rho goes there
+
+    // ---- psi, rho (hi / lo bf16 into the q tile), partial z
+    uint16_t* rh = reinterpret_cast<uint16_t*>(sq);
+    uint16_t* rl = reinterpret_cast<uint16_t*>(sq + Ly::RHO_BYTES);
+    float zp[NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) zp[j][0] = zp[j][1] = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int row = warp * 16 + g + half * 8;
+      const int tok = tok0 + row;
+      const bool vok = row < valid;
+      const int pt = tok / (p.Hg * p.W), py = (tok / p.W) % p.Hg, px = tok % p.W;
+#pragma unroll
+      for (int nj = 0; nj < NT; ++nj) {
+        const int col = nj * 8 + 2 * t4;
+        const int pr = col >> 1;
+        const float p0 = vok ? phi(acc[nj][2 * half]) : 0.f;
+        const float p1 = vok ? phi(acc[nj][2 * half + 1]) : 0.f;
+        zp[nj][0] += p0;
+        zp[nj][1] += p1;
+        const int ax = p.rope.axis[pr];
+        const int pos = ax == 0 ? pt : (ax == 1 ? py : px);
+        float sn, cs;
+        if (p.tab_entries) {
+          const float2 v = M.tab[p.tab_base[pr] + pos * p.tab_stride[pr]];
+          cs = v.x;
+          sn = v.y;
+        } else {
+          rope_sincos(pos, p.rope.freq[pr], &sn, &cs);
+        }
+        const float r0 = p0 * cs - p1 * sn, r1 = p0 * sn + p1 * cs;
+        const uint32_t hi = pack_bf16(r0, r1);
+        const uint32_t lo = pack_bf16(r0 - bf16_lo(hi), r1 - bf16_hi(hi));
+        *reinterpret_cast<uint32_t*>(rh + row * Ly::PS + col) = hi;
+        *reinterpret_cast<uint32_t*>(rl + row * Ly::PS + col) = lo;
+      }
+    }
+#pragma unroll
+    for (int nj = 0; nj < NT; ++nj)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float x = zp[nj][e];
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        x += __shfl_xor_sync(0xffffffffu, x, 8);
+        x += __shfl_xor_sync(0xffffffffu, x, 16);
+        if (g == 0) M.zpart[warp][nj * 8 + 2 * t4 + e] = x;
+      }
+    __syncthreads();
+    const size_t state = bh * p.nb + blk;
+    if (tid < R) {
+      float z = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) z += M.zpart[w][tid];
+      p.z_blk[state * R + tid] = z;
+    }
+
+    // ---- S_j^T pieces: C[r, d] = rho^T V, warp w owns d columns [16w, 16w + 16)
+    {
+      constexpr int MT = R / 16;
+      float c2[MT][2][4];
+#pragma unroll
+      for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) c2[i][j][e] = 0.f;
+      const uint32_t rhb = smem_u32(rh), rlb = smem_u32(rl), vb = smem_u32(sv);
+#pragma unroll
+      for (int kt = 0; kt < BS; kt += 16) {
+        const int arow = kt + (lane & 7) + ((lane >> 4) << 3);
+        const int acol = ((lane >> 3) & 1) * 8;
+        uint32_t bb[4];
+        ldsm_x4_t(bb, vb + sw_off(kt + (lane & 15), warp * 16 + (lane >> 4) * 8));
+#pragma unroll
+        for (int mi = 0; mi < MT; ++mi) {
+          uint32_t ah[4], al[4];
+          ldsm_x4_t(ah, rhb + (arow * Ly::PS + mi * 16 + acol) * 2);
+          ldsm_x4_t(al, rlb + (arow * Ly::PS + mi * 16 + acol) * 2);
+          mma16816(c2[mi][0], ah, bb[0], bb[1]);
+          mma16816(c2[mi][0], al, bb[0], bb[1]);
+          mma16816(c2[mi][1], ah, bb[2], bb[3]);
+          mma16816(c2[mi][1], al, bb[2], bb[3]);
+        }
+      }
+      float* Sout = p.S_blk + state * R * D;
+#pragma unroll
+      for (int mi = 0; mi < MT; ++mi)
+#pragma unroll
+        for (int nj = 0; nj < 2; ++nj) {
+          const int rr = mi * 16 + g, dd = warp * 16 + nj * 8 + 2 * t4;
+          *reinterpret_cast<float2*>(Sout + (size_t)rr * D + dd) = make_float2(c2[mi][nj][0], c2[mi][nj][1]);
+          *reinterpret_cast<float2*>(Sout + (size_t)(rr + 8) * D + dd) =
+              make_float2(c2[mi][nj][2], c2[mi][nj][3]);
+        }
+    }
+    __syncthreads();  // stage st is free for item it + 2
+  }
+  // drain: if we stopped early, let the copies in flight land before exiting
+  if (tid == 0) {
+    int no_abort = 0;
+    for (int j = it; j < my_items && j <= it + 1; ++j) mbar_wait(&M.full[j & 1], (j >> 1) & 1, &no_abort);
+  }
+  if (tid == 0 && M.abort && p.dev_err) atomicOr(p.dev_err, ROLA_DEVERR_TIMEOUT);
+}
+
+template <int R>
+static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            Params prm, cudaStream_t cs) {
+  using Ly = Layout<R>;
+  CUtensorMap mq, mk, mv;
+  if (!rola_host::make_act_map(&mk, k, s, BS) || !rola_host::make_act_map(&mv, v, s, BS) ||
+      !rola_host::make_act_map(&mq, q ? q : k, s, BS))
+    return ROLA_ERR_CUDA;
+  const size_t smem = Ly::misc_off + sizeof(Misc) + 1024;
+  auto kern = rola_prep_kernel<R>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return ROLA_ERR_CUDA;
+  const int nsm = rola_host::sm_count();
+  const int grid = prm.items < nsm ? prm.items : nsm;
+  kern<<<grid, kThreads, smem, cs>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+}
+
+}  // namespace prep
+
+bool prep_kernel_supports(const rola_shape_t* s) {
+  return s->d == 128 && s->block == 128 && (s->r == 16 || s->r == 32);
+}
+
+// Block means (if q, qbar and kbar are given) and block states of every
+// (batch, head, block); d = 128 and 128-token blocks.
+rola_status_t launch_prep_kernel(const rola_shape_t* s, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const uint16_t* P, double* qbar, double* kbar,
+                                 float* S_blk, float* z_blk, int32_t* dev_err, cudaStream_t cs) {
+  prep::Params prm{};
+  prm.B = s->B;
+  prm.H = s->H;
+  prm.N = s->N;
+  prm.nb = rola_num_blocks(s);
+  prm.Hg = s->Hg;
+  prm.W = s->W;
+  prm.items = s->B * s->H * prm.nb;
+  prm.do_pool = (q && qbar && kbar) ? 1 : 0;
+  prm.qbar = qbar;
+  prm.kbar = kbar;
+  prm.P = P;
+  prm.S_blk = S_blk;
+  prm.z_blk = z_blk;
+  prm.dev_err = dev_err;
+  rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
+  rola_host::RopeTabLayout tl;
+  rola_host::rope_table_layout(s, prm.rope.axis, &tl);
+  for (int i = 0; i < 16; ++i) {
+    prm.tab_base[i] = tl.base[i];
+    prm.tab_stride[i] = tl.stride[i];
+  }
+  for (int i = 0; i < 17; ++i) prm.tab_first[i] = tl.first[i];
+  prm.tab_entries = tl.entries <= prep::kTabCap ? tl.entries : 0;
+  if (s->r == 32) return prep::launch<32>(s, q, k, v, prm, cs);
+  return prep::launch<16>(s, q, k, v, prm, cs);
+}
+
+}  // namespace rola

@@ -156,33 +156,44 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ si
     const int j = i * 32 + lane;
     v[i] = (i < nper && j < nb) ? s[j] : -DBL_MAX;
   }
+  constexpr int kNone = 0x7fffffff;
   uint32_t taken = 0;
+  // this lane's best untaken candidate (largest score, then lowest index)
+  auto local_best = [&](double& best, int& bidx) {
+    best = -INFINITY;
+    bidx = kNone;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int j = i * 32 + lane;
+      if (i < nper && j < nb && !((taken >> i) & 1u) && (bidx == kNone || v[i] > best)) {
+        best = v[i];
+        bidx = j;
+      }
+    }
+  };
   if (kb >= nb) {
     taken = 0xffffffffu;
   } else {
+    double lb;
+    int li;
+    local_best(lb, li);
     for (int round = 0; round < kb; ++round) {
-      double best = -INFINITY;
-      int bidx = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < kMaxPerLane; ++i) {
-        const int j = i * 32 + lane;
-        if (i < nper && j < nb && !((taken >> i) & 1u) && (v[i] > best || bidx == 0x7fffffff)) {
-          if (bidx == 0x7fffffff || v[i] > best) {
-            best = v[i];
-            bidx = j;
-          }
-        }
-      }
+      double best = lb;
+      int bidx = li;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
         const double ob = __shfl_xor_sync(0xffffffffu, best, off);
         const int oi = __shfl_xor_sync(0xffffffffu, bidx, off);
-        if (oi != 0x7fffffff && (bidx == 0x7fffffff || ob > best || (ob == best && oi < bidx))) {
+        if (oi != kNone && (bidx == kNone || ob > best || (ob == best && oi < bidx))) {
           best = ob;
           bidx = oi;
         }
       }
-      if (bidx != 0x7fffffff && (bidx & 31) == lane) taken |= 1u << (bidx >> 5);
+      // only the lane that owned the winner needs a new candidate
+      if (bidx != kNone && (bidx & 31) == lane) {
+        taken |= 1u << (bidx >> 5);
+        local_best(lb, li);
+      }
     }
   }
   int pos = 0;
@@ -193,6 +204,17 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ si
     if (mine) out[pos + __popc(ball & ((1u << lane) - 1u))] = j;
     pos += __popc(ball);
   }
+}
+
+// Scores and top-k from pooled block means (float64 [B, H, nb, d]).
+rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, const double* kbar,
+                                 double* sigma, int32_t* idx, cudaStream_t cs) {
+  const int nb = rola_num_blocks(s);
+  const int tiles = (nb + kScTile - 1) / kScTile;
+  score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, 0, cs>>>(qbar, kbar, sigma, s->H, s->d, nb);
+  const int rows = s->B * s->H * nb;
+  topk_kernel<<<(rows + 7) / 8, 256, 0, cs>>>(sigma, idx, rows, nb, s->k_b);
+  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 
 }  // namespace rola
@@ -229,9 +251,6 @@ extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_
   if (scores_opt) sig = scores_opt;
 
   pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
-  const int tiles = (nb + kScTile - 1) / kScTile;
-  score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, 0, cs>>>(qbar, kbar, sig, s->H, s->d, nb);
-  const int rows = s->B * s->H * nb;
-  topk_kernel<<<(rows + 7) / 8, 256, 0, cs>>>(sig, idx, rows, nb, s->k_b);
-  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return ROLA_ERR_CUDA;
+  return select_from_pooled(s, qbar, kbar, sig, idx, cs);
 }

@@ -249,6 +249,15 @@ static rola_status_t launch_states(const rola_shape_t* s, const uint16_t* k, con
   return ROLA_OK;
 }
 
+rola_status_t launch_states_total(const rola_shape_t* s, const float* S_blk, const float* z_blk,
+                                  float* S_glb, float* z_glb, cudaStream_t cs) {
+  const int nb = rola_num_blocks(s);
+  const int rd = s->r * s->d;
+  states_total_kernel<<<dim3((rd + s->r + 255) / 256, s->B * s->H), 256, 0, cs>>>(S_blk, z_blk, S_glb,
+                                                                                  z_glb, nb, rd, s->r);
+  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+}
+
 }  // namespace rola
 
 using namespace rola;
@@ -265,6 +274,12 @@ extern "C" rola_status_t rola_block_states(const rola_shape_t* s, const uint16_t
       !rola_host::aligned(S_glb, 4) || !rola_host::aligned(z_glb, 4))
     return ROLA_ERR_ALIGNMENT;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (prep_kernel_supports(s)) {
+    // the persistent TMA-fed pass (no pooling)
+    st = launch_prep_kernel(s, nullptr, k, v, P, nullptr, nullptr, S_blk, z_blk, nullptr, cs);
+    if (st != ROLA_OK) return st;
+    return launch_states_total(s, S_blk, z_blk, S_glb, z_glb, cs);
+  }
   RopeTable rope{};
   rola_host::rope_frequencies(s->r, s->rope_base, rope.freq, rope.axis);
   const int key = s->d * 1000000 + s->r * 1000 + s->block;
@@ -280,9 +295,5 @@ extern "C" rola_status_t rola_block_states(const rola_shape_t* s, const uint16_t
     default: return ROLA_ERR_UNSUPPORTED;
   }
   if (st != ROLA_OK) return st;
-  const int nb = rola_num_blocks(s);
-  const int rd = s->r * s->d;
-  states_total_kernel<<<dim3((rd + s->r + 255) / 256, s->B * s->H), 256, 0, cs>>>(
-      S_blk, z_blk, S_glb, z_glb, nb, rd, s->r);
-  return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+  return launch_states_total(s, S_blk, z_blk, S_glb, z_glb, cs);
 }

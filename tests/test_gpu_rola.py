@@ -219,3 +219,10 @@ def test_layer_entry_points(cfg):
     hl(*host, out_h)
     torch.cuda.synchronize()
     assert torch.equal(out_h, out.cpu())
+    # timed variant: same result, ordered positive stage times
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    out3 = layer(q, k, v, P, gate, events=ev)
+    torch.cuda.synchronize()
+    assert torch.equal(out3, out)
+    assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0
+    assert rb.layer_launches(shape) in (5, 6)
