@@ -211,19 +211,26 @@ rola_status_t fp8_quantize_weight(int32_t N, int32_t K, const float* w, uint8_t*
 
 /* y[m,n] = bf16( (sum_k dec(x_q[m,k]) dec(w_q[n,k])) * x_scale[m] * w_scale[n] )
  * on the tensor cores (tcgen05 kind::f8f6f4, fp32 accumulation in tensor
- * memory).  x_q [M, K], w_q [N, K] row-major E4M3 bytes, y [M, N] bf16.
- * K and N multiples of 128; all pointers 16-byte aligned. */
+ * memory); write-up section 07 (W8A8 FP8 E4M3 projections).
+ * x_q [M, K], w_q [N, K] row-major E4M3 bytes (both K-major), x_scale [M],
+ * w_scale [N] float32, y [M, N] row-major bf16; all device pointers, owned by
+ * the caller.  N a multiple of 32, K a multiple of 16 (a K tail inside the
+ * last 128-wide slice is zero-padded by the copy engine).  x_q, w_q, y and
+ * w_scale 16-byte aligned, x_scale 4-byte aligned.  Asynchronous on `stream`.
+ * dev_err: optional device int32 that receives ROLA_DEVERR_TIMEOUT if a
+ * pipeline wait ran out (y is then incomplete). */
 rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
                             const float* x_scale, const uint8_t* w_q, const float* w_scale,
-                            uint16_t* y, void* stream);
+                            uint16_t* y, int32_t* dev_err, void* stream);
 
 /* Workspace of fp8_linear_w8a8: the quantised activations and their scales. */
 size_t fp8_linear_workspace_bytes(int32_t M, int32_t K);
 
-/* x (bf16 [M, K]) -> per-token quantisation into ws -> fp8_gemm_w8a8. */
+/* x (bf16 [M, K]) -> per-token quantisation into ws -> fp8_gemm_w8a8.
+ * Same constraints as the two calls; dev_err as in fp8_gemm_w8a8. */
 rola_status_t fp8_linear_w8a8(int32_t M, int32_t N, int32_t K, const uint16_t* x,
                               const uint8_t* w_q, const float* w_scale, uint16_t* y, void* ws,
-                              size_t ws_bytes, void* stream);
+                              size_t ws_bytes, int32_t* dev_err, void* stream);
 
 #ifdef __cplusplus
 }

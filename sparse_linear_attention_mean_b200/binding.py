@@ -113,11 +113,11 @@ def lib() -> ctypes.CDLL:
         L.fp8_quantize_weight.restype = ctypes.c_int
         L.fp8_quantize_weight.argtypes = [i32, i32, vp, vp, vp, vp]
         L.fp8_gemm_w8a8.restype = ctypes.c_int
-        L.fp8_gemm_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.fp8_gemm_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
         L.fp8_linear_workspace_bytes.restype = sz
         L.fp8_linear_workspace_bytes.argtypes = [i32, i32]
         L.fp8_linear_w8a8.restype = ctypes.c_int
-        L.fp8_linear_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.fp8_linear_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
         _lib = L
     return _lib
 
@@ -325,7 +325,7 @@ def fp8_quantize_weight(w, *, stream=None):
     return wq, sc
 
 
-def fp8_gemm(xq, xs, wq, ws, *, out=None, stream=None):
+def fp8_gemm(xq, xs, wq, ws, *, out=None, dev_err=None, stream=None):
     M, K = xq.shape
     N = wq.shape[0]
     _need(xq, torch.uint8, (M, K), "x_q")
@@ -336,11 +336,11 @@ def fp8_gemm(xq, xs, wq, ws, *, out=None, stream=None):
         out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
     _need(out, torch.bfloat16, (M, N), "y")
     _check(lib().fp8_gemm_w8a8(M, N, K, _ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(out),
-                               _stream(stream)), "fp8_gemm_w8a8")
+                               _ptr(dev_err), _stream(stream)), "fp8_gemm_w8a8")
     return out
 
 
-def fp8_linear(x, wq, ws, *, out=None, workspace=None, stream=None):
+def fp8_linear(x, wq, ws, *, out=None, workspace=None, dev_err=None, stream=None):
     M, K = x.shape
     N = wq.shape[0]
     _need(x, torch.bfloat16, (M, K), "x")
@@ -352,5 +352,5 @@ def fp8_linear(x, wq, ws, *, out=None, workspace=None, stream=None):
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _check(lib().fp8_linear_w8a8(M, N, K, _ptr(x), _ptr(wq), _ptr(ws), _ptr(out), _ptr(workspace),
-                                 nbytes, _stream(stream)), "fp8_linear_w8a8")
+                                 nbytes, _ptr(dev_err), _stream(stream)), "fp8_linear_w8a8")
     return out

@@ -116,14 +116,6 @@ extern "C" rola_status_t fp8_quantize_weight(int32_t N, int32_t K, const float* 
   return launch_quant<float>(N, K, w, w_q, w_scale, reinterpret_cast<cudaStream_t>(stream));
 }
 
-extern "C" rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
-                                       const float* x_scale, const uint8_t* w_q,
-                                       const float* w_scale, uint16_t* y, void* stream) {
-  (void)M; (void)N; (void)K; (void)x_q; (void)x_scale; (void)w_q; (void)w_scale; (void)y;
-  (void)stream;
-  return ROLA_ERR_UNSUPPORTED;
-}
-
 extern "C" size_t fp8_linear_workspace_bytes(int32_t M, int32_t K) {
   if (M < 1 || K < 1) return 0;
   return rola_internal::round_up((size_t)M * K, 256) + rola_internal::round_up((size_t)M * 4, 256);
@@ -131,7 +123,7 @@ extern "C" size_t fp8_linear_workspace_bytes(int32_t M, int32_t K) {
 
 extern "C" rola_status_t fp8_linear_w8a8(int32_t M, int32_t N, int32_t K, const uint16_t* x,
                                          const uint8_t* w_q, const float* w_scale, uint16_t* y,
-                                         void* ws, size_t ws_bytes, void* stream) {
+                                         void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
   if (M < 1 || N < 1 || K < 1 || !x || !w_q || !w_scale || !y) return ROLA_ERR_INVALID_ARG;
   const size_t need = fp8_linear_workspace_bytes(M, K);
   if (!ws || ws_bytes < need || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
@@ -139,5 +131,5 @@ extern "C" rola_status_t fp8_linear_w8a8(int32_t M, int32_t N, int32_t K, const 
   float* xs = reinterpret_cast<float*>(xq + rola_internal::round_up((size_t)M * K, 256));
   rola_status_t st = fp8_quantize_rows_bf16(M, K, x, xq, xs, stream);
   if (st != ROLA_OK) return st;
-  return fp8_gemm_w8a8(M, N, K, xq, xs, w_q, w_scale, y, stream);
+  return fp8_gemm_w8a8(M, N, K, xq, xs, w_q, w_scale, y, dev_err, stream);
 }

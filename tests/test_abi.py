@@ -78,3 +78,16 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.rola_block_states(ctypes.byref(cs), odd, ok, ok, ok, ok, ok, ok, None) == 5
     assert lib.rola_select_blocks(ctypes.byref(cs), ok, ok, ok, None, None, 0, None) == 3  # no workspace
     assert lib.fp8_quantize_rows_bf16(4, 15, ok, ok, ok, None) == 1                          # K % 16
+
+
+def test_fp8_gemm_arguments_rejected_on_host(lib):
+    ok = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4104)  # 8-byte aligned only
+    gemm = lib.fp8_gemm_w8a8
+    assert gemm(64, 40, 64, ok, ok, ok, ok, ok, None, None) == 1    # N % 32
+    assert gemm(64, 64, 24, ok, ok, ok, ok, ok, None, None) == 1    # K % 16
+    assert gemm(0, 64, 64, ok, ok, ok, ok, ok, None, None) == 1     # empty M
+    assert gemm(64, 64, 64, None, ok, ok, ok, ok, None, None) == 1  # null operand
+    assert gemm(64, 64, 64, odd, ok, ok, ok, ok, None, None) == 5   # misaligned codes
+    assert gemm(64, 64, 64, ok, ok, ok, odd, ok, None, None) == 5   # misaligned w_scale
+    assert lib.fp8_linear_w8a8(64, 64, 64, ok, ok, ok, ok, None, 0, None, None) == 3  # no workspace

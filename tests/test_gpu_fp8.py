@@ -1,0 +1,140 @@
+"""GPU parity of the W8A8 FP8 E4M3 projections against the oracle, through the
+C ABI (SparkDiffusion write-up, section 07).
+
+* quantisation: E4M3 codes and float32 scales bit-exact (the oracle rounds
+  the reciprocal and the product to float32 as the kernel does);
+* GEMM: relative Frobenius error <= 1e-2 against the oracle's float64 product
+  of the same codes; per element within 1e-2 |ref| plus 1e-3 of the row's
+  largest magnitude (bf16 output rounding, fp32 accumulation order).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import fp8_oracle as fo
+from sparse_linear_attention_mean_b200 import binding as rb
+from sparse_linear_attention_mean_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+FROB = 1e-2
+
+
+def _bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
+
+
+def _bf16_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def _check_gemm(y_dev, ref, what):
+    y = y_dev.float().cpu().numpy().astype(np.float64)
+    fro = np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300)
+    assert fro <= FROB, f"{what}: relative Frobenius {fro:.3g}"
+    bound = 1e-2 * np.abs(ref) + 1e-3 * np.abs(ref).max(axis=1, keepdims=True)
+    bad = np.abs(y - ref) > bound
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements out of tolerance"
+    return fro
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (37, 80), (256, 5120), (300, 1040)])
+def test_quantize_rows_bitexact(M, K):
+    bits = synth.make_normal_bf16((M, K), seed=M * 7 + K, stream=1, std=3.0)
+    if M > 2:
+        bits[2] = 0          # an all-zero row takes scale 1
+        bits[1, 5] = 0x4380  # 256.0: a large outlier in one row
+    xq, xs = rb.fp8_quantize_rows(_bf16_dev(bits))
+    codes, scale = fo.quantize_rows(_bf16_f32(bits))
+    torch.cuda.synchronize()
+    assert np.array_equal(xq.cpu().numpy(), codes)
+    assert np.array_equal(xs.cpu().numpy(), scale)
+
+
+@pytest.mark.parametrize("N,K", [(96, 48), (512, 5120)])
+def test_quantize_weight_bitexact(N, K):
+    w = (synth.make_normal_bf16((N, K), seed=N + K, stream=2).astype(np.uint32) << 16).view(np.float32)
+    w = np.ascontiguousarray(w * np.float32(0.013))
+    wq, ws = rb.fp8_quantize_weight(torch.from_numpy(w).cuda())
+    codes, scale = fo.quantize_rows(w)
+    torch.cuda.synchronize()
+    assert np.array_equal(wq.cpu().numpy(), codes)
+    assert np.array_equal(ws.cpu().numpy(), scale)
+
+
+def _random_codes(shape, seed):
+    """Finite E4M3 codes (0x7f / 0xff are NaN and never produced by the cast)."""
+    g = np.random.default_rng(seed)
+    c = g.integers(0, 256, size=shape, dtype=np.uint8)
+    return np.where((c & 0x7f) == 0x7f, c ^ 0x01, c).astype(np.uint8)
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 32, 16),        # single row, one 32-column chunk, K inside one slice
+    (200, 96, 80),      # ragged M tile, partial N tile, K tail
+    (128, 256, 128),    # exactly one tile
+    (1000, 768, 1024),  # several tiles in both directions, several K slices
+    (333, 544, 2064),   # ragged everything, more tiles than one pass of the CTAs
+])
+def test_gemm_small(M, N, K):
+    xq = _random_codes((M, K), 11 + M)
+    wq = _random_codes((N, K), 13 + N)
+    g = np.random.default_rng(M + N + K)
+    xs = g.uniform(0.001, 0.02, size=M).astype(np.float32)
+    ws = g.uniform(0.001, 0.02, size=N).astype(np.float32)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = rb.fp8_gemm(torch.from_numpy(xq).cuda(), torch.from_numpy(xs).cuda(),
+                    torch.from_numpy(wq).cuda(), torch.from_numpy(ws).cuda(), dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    _check_gemm(y, fo.gemm_w8a8(xq, xs, wq, ws), f"gemm {M}x{N}x{K}")
+
+
+def test_gemm_rejects_bad_shapes():
+    xq = torch.zeros((4, 64), dtype=torch.uint8, device="cuda")
+    xs = torch.ones(4, device="cuda")
+    for N, K in ((40, 64), (64, 24)):  # N % 32, K % 16
+        wq = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
+        with pytest.raises(rb.RolaError):
+            rb.fp8_gemm(torch.zeros((4, K), dtype=torch.uint8, device="cuda"), xs, wq,
+                        torch.ones(N, device="cuda"))
+
+
+_BLOCK = {}
+
+
+def _block_inputs():
+    if not _BLOCK:
+        w = synth.WORKLOADS[4]
+        _BLOCK["w"] = w
+        _BLOCK["inp"] = synth.make_block_inputs(w)
+    return _BLOCK["w"], _BLOCK["inp"]
+
+
+def test_linear_full_size_sampled():
+    """Full 14B-720P projection (x [75600, 5120] -> [75600, 5120]) in the
+    launch configuration the benchmark times; the oracle checks sampled rows,
+    including the ragged last tile, against every output column."""
+    w, inp = _block_inputs()
+    D = w.model_dim
+    x = _bf16_dev(inp["x"])
+    Wq = np.ascontiguousarray(inp["Wq"])
+    wq, ws = rb.fp8_quantize_weight(torch.from_numpy(Wq).cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = rb.fp8_linear(x, wq, ws, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    M = x.shape[0]
+    rows = np.unique(np.concatenate([np.arange(0, 8), np.arange(M - 80, M, 9), [M - 1],
+                                     np.random.default_rng(5).integers(0, M, 24)]))
+    xs_codes, xs_scale = fo.quantize_rows(_bf16_f32(inp["x"][rows]))
+    w_codes, w_scale = fo.quantize_rows(Wq)
+    assert np.array_equal(wq.cpu().numpy(), w_codes)
+    ref = fo.gemm_w8a8(xs_codes, xs_scale, w_codes, w_scale)
+    _check_gemm(y[torch.from_numpy(rows).cuda()], ref, "linear 75600x5120x5120")
+    # the fused call equals quantisation followed by the GEMM
+    xq, xsc = rb.fp8_quantize_rows(x)
+    y2 = rb.fp8_gemm(xq, xsc, wq, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    assert D == 5120
