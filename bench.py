@@ -241,6 +241,12 @@ def run_gpu(args) -> int:
     flop = w.sparse_flops()
     value = world * flop * K / (total_ms * 1e-3) / 1e12
 
+    # one FP8 W8A8 projection of the full attention block (x [N, 5120] ->
+    # [N, 5120]: quantisation + tcgen05 GEMM), timed on its own after the layer
+    fp8 = None
+    if not args.no_fp8 and w.H * w.d == 5120:
+        fp8 = fp8_projection(w.B * w.N, w.H * w.d, stream)
+
     # end to end through the host-buffer entry point (pinned host memory)
     e2e = None
     if not args.no_e2e:
@@ -290,6 +296,7 @@ def run_gpu(args) -> int:
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                          "peak_source": peaks["source"] + " bf16 burst"},
             "e2e": e2e,
+            "fp8_projection": fp8,
             "gpu_launches": K * launches_per_step,
             "clocks": clk.summary(),
         }
@@ -300,6 +307,46 @@ def run_gpu(args) -> int:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def fp8_projection(M: int, D: int, stream, reps: int = 5) -> dict:
+    """Times fp8_linear_w8a8 (per-token quantisation + W8A8 GEMM) for x [M, D]
+    bf16 ~ N(0, 1) and W [D, D] ~ N(0, 1/D), and the GEMM alone."""
+    import torch
+    from sparse_linear_attention_mean_b200 import binding as rb
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4)
+    x = torch.randn((M, D), generator=g, device="cuda").to(torch.bfloat16)
+    W = torch.randn((D, D), generator=g, device="cuda") / D ** 0.5
+    wq, ws = rb.fp8_quantize_weight(W)
+    xq, xs = rb.fp8_quantize_rows(x)
+    y = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws_buf = torch.empty(rb.lib().fp8_linear_workspace_bytes(M, D), dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    gemm_ms = timed(lambda: rb.fp8_gemm(xq, xs, wq, ws, out=y, dev_err=err, stream=stream))
+    lin_ms = timed(lambda: rb.fp8_linear(x, wq, ws, out=y, workspace=ws_buf, dev_err=err, stream=stream))
+    assert int(err.item()) == 0
+    flop = 2.0 * M * D * D
+    peaks = measured_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    return {"shape_mnk": [M, D, D], "gemm_ms": gemm_ms, "linear_ms": lin_ms,
+            "gemm_tflops": flop / gemm_ms / 1e9, "linear_tflops": flop / lin_ms / 1e9,
+            "fp8_peak_tflops": fp8_peak,
+            "peak_source": peaks["source"] + " bf16 burst x 2 (nominal fp8:bf16 ratio)",
+            "gemm_frac": flop / gemm_ms / 1e9 / fp8_peak}
 
 
 def kernel_hash() -> str:
@@ -319,6 +366,7 @@ def main() -> int:
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling runs)")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projection timing")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
                     help="attention workload id of synth.WORKLOADS (profiling of smaller cases)")
     args = ap.parse_args()

@@ -138,3 +138,79 @@ def test_linear_full_size_sampled():
     torch.cuda.synchronize()
     assert torch.equal(y, y2)
     assert D == 5120
+
+
+def _oracle_head_projections(x_bits, Ws, heads, d, chunk=4096):
+    """The oracle's W8A8 projections of x by each weight of `Ws`, restricted to
+    the output columns of `heads` and rounded to bf16 as the projections'
+    outputs are; a list of uint16 bit arrays [M, len(heads), d]."""
+    cols = np.concatenate([np.arange(h * d, (h + 1) * d) for h in heads])
+    wd, wsc = [], []
+    for W in Ws:
+        w_codes, w_scale = fo.quantize_rows(np.ascontiguousarray(W))
+        wd.append(fo.e4m3_decode(w_codes[cols]))
+        wsc.append(w_scale[cols].astype(np.float64))
+    wd, wsc = np.concatenate(wd), np.concatenate(wsc)
+    out = np.empty((x_bits.shape[0], wd.shape[0]), dtype=np.float64)
+
+    def rows(m0):
+        xc, xs = fo.quantize_rows(_bf16_f32(x_bits[m0:m0 + chunk]))
+        out[m0:m0 + chunk] = (fo.e4m3_decode(xc) @ wd.T) * xs[:, None].astype(np.float64) * wsc[None, :]
+
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        list(ex.map(rows, range(0, x_bits.shape[0], chunk)))
+    bits = synth.f32_to_bf16_bits(out.astype(np.float32))
+    n = len(cols)
+    return [bits[:, i * n:(i + 1) * n].reshape(x_bits.shape[0], len(heads), d).copy()
+            for i in range(len(Ws))]
+
+
+def test_attention_block_chain():
+    """The full 14B-720P attention block: FP8 QKV projections -> RoLA layer ->
+    FP8 output projection, all on the GPU.  The oracle runs the same chain for
+    two heads from x on its own (projection of those heads' columns, mask,
+    attention at sampled query blocks, given the oracle's mask)."""
+    from oracle import rola_oracle as ro
+    from helpers import check_close, mask_mismatch
+    w, inp = _block_inputs()
+    D, H, d = w.model_dim, w.H, w.d
+    shape = rb.Shape.of(w)
+    x = _bf16_dev(inp["x"])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    proj = {}
+    for nm in ("Wq", "Wk", "Wv"):
+        wq, ws = rb.fp8_quantize_weight(torch.from_numpy(np.ascontiguousarray(inp[nm])).cuda())
+        proj[nm] = rb.fp8_linear(x, wq, ws, dev_err=err).view(w.B, w.N, H, d)
+    P = torch.from_numpy(np.ascontiguousarray(inp["P"])).view(torch.bfloat16).cuda()
+    gate = torch.from_numpy(inp["gate"]).cuda()
+    q, k, v = proj["Wq"], proj["Wk"], proj["Wv"]
+    idx_gpu = rb.select_blocks(shape, q, k)
+    heads = [0, H - 1]
+    oq, ok_, ov = _oracle_head_projections(inp["x"], [inp["Wq"], inp["Wk"], inp["Wv"]], heads, d)
+    sub = {"q": oq[None], "k": ok_[None], "v": ov[None],
+           "P": np.ascontiguousarray(inp["P"][heads]), "gate": inp["gate"][heads]}
+    idx_ref, sig = ro.select_all(sub, w.block, w.k_b)
+    torch.cuda.synchronize()
+    # the GPU's own mask from its own projections: near-tie rows may differ
+    ties, bad = mask_mismatch(idx_gpu[:, heads].cpu().numpy(), idx_ref, sig, w.k_b)
+    assert not bad, f"mask rows differ outside near-ties: {bad[:5]}"
+    # attention given the oracle's mask for the checked heads
+    idx_full = idx_gpu.clone()
+    idx_full[:, heads] = torch.from_numpy(idx_ref).cuda()
+    states = rb.block_states(shape, k, v, P)
+    o = rb.attention_fwd(shape, q, k, v, idx_full, P, states, gate, dev_err=err)
+    nb = w.n_blocks
+    qblocks = [0, nb // 2, nb - 1]
+    res = ro.rola_forward(sub, bs=w.block, k_b=w.k_b, grid=(w.T, w.Hg, w.W), rope_base=w.rope_base,
+                          idx=idx_ref, qblocks=qblocks)
+    wo_q, wo_s = rb.fp8_quantize_weight(torch.from_numpy(np.ascontiguousarray(inp["Wo"])).cuda())
+    y = rb.fp8_linear(o.view(w.B * w.N, D), wo_q, wo_s, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    o64 = o.float().cpu().numpy().astype(np.float64)
+    for (b, j), r in res.items():
+        for a, rows in r.o.items():
+            lo, hi = ro.block_range(a, w.block, w.N)
+            check_close(o64[b, lo:hi, heads[j], :], rows, what=f"head {heads[j]} block {a}")
+    assert torch.isfinite(y.float()).all()
