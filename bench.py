@@ -197,6 +197,8 @@ def run_gpu(args) -> int:
                                 device_id=torch.device("cuda", local))
 
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        w = synth.custom_workload(w, H=args.heads)
     shape = rb.Shape.of(w)
     inp = synth.make_inputs(w)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
@@ -367,6 +369,8 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projection timing")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (per-head work unchanged; for profiling captures)")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
                     help="attention workload id of synth.WORKLOADS (profiling of smaller cases)")
     args = ap.parse_args()

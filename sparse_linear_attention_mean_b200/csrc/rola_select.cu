@@ -136,44 +136,109 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
 }
 
 // ---------------------------------------------------------------- top-k
-// One warp per (b, h, query block).  Lane l holds scores of blocks l, l+32, ...
-// (n_blocks <= 32 * 32).  k_b rounds of a warp arg-max by (score desc, index
-// asc); the chosen set is then written in ascending block order.
+// One warp per (b, h, query block).  Lane l holds the scores of blocks l,
+// l + 32, ... (MAXP per lane, n_blocks <= 32 * MAXP).  Order: score
+// descending, then block index ascending.
+//
+// Fast path (k_b <= 32, k_b < n_blocks): the k_b-th largest of the 32 lane
+// maxima, T, is a lower bound of the k_b-th largest score (k_b lanes hold a
+// score >= T), so the kept set lies among the scores >= T.  Those candidates
+// (typically a few dozen) go to shared memory and each one's exact rank is
+// counted against the others; rank < k_b is kept.  With more than kCandCap
+// candidates, or a larger k_b, the warp falls back to k_b rounds of a warp
+// arg-max.  The kept set is written in ascending block order.
 constexpr int kMaxPerLane = 32;
+constexpr int kCandCap = 256;
+constexpr int kTopkWarps = 8;
 
-__global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ sigma,
-                                                   int32_t* __restrict__ idx, int rows, int nb,
-                                                   int kb) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= rows) return;
+template <int MAXP>
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const double* __restrict__ sigma,
+                                                               int32_t* __restrict__ idx, int rows,
+                                                               int nb, int kb) {
+  __shared__ double cand_v[kTopkWarps][kCandCap];
+  __shared__ int cand_j[kTopkWarps][kCandCap];
+  __shared__ uint32_t kept_bits[kTopkWarps][32];
+  const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = blockIdx.x * kTopkWarps + wib;
+  if (warp >= rows) return;  // uniform per warp
   const double* s = sigma + (size_t)warp * nb;
   int32_t* out = idx + (size_t)warp * kb;
-  const int nper = (nb + 31) / 32;
-  double v[kMaxPerLane];
+  double v[MAXP];
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < MAXP; ++i) {
     const int j = i * 32 + lane;
-    v[i] = (i < nper && j < nb) ? s[j] : -DBL_MAX;
+    v[i] = j < nb ? s[j] : -INFINITY;
   }
   constexpr int kNone = 0x7fffffff;
   uint32_t taken = 0;
-  // this lane's best untaken candidate (largest score, then lowest index)
-  auto local_best = [&](double& best, int& bidx) {
-    best = -INFINITY;
-    bidx = kNone;
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-      const int j = i * 32 + lane;
-      if (i < nper && j < nb && !((taken >> i) & 1u) && (bidx == kNone || v[i] > best)) {
-        best = v[i];
-        bidx = j;
-      }
-    }
-  };
+  bool done = false;
   if (kb >= nb) {
     taken = 0xffffffffu;
-  } else {
+    done = true;
+  } else if (kb <= 32) {
+    double m = v[0];
+#pragma unroll
+    for (int i = 1; i < MAXP; ++i) m = fmax(m, v[i]);
+    // rank of this lane's maximum among the 32 (value desc, lane asc)
+    int rank = 0;
+#pragma unroll
+    for (int l2 = 0; l2 < 32; ++l2) {
+      const double o = __shfl_sync(0xffffffffu, m, l2);
+      rank += (o > m || (o == m && l2 < lane)) ? 1 : 0;
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, rank == kb - 1);
+    const double T = __shfl_sync(0xffffffffu, m, __ffs(who) - 1);
+    // gather the candidates (finite: at least k_b lanes hold a real score)
+    int C = 0;
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < MAXP; ++i) {
+      const int j = i * 32 + lane;
+      const bool c = j < nb && v[i] >= T;
+      const uint32_t ball = __ballot_sync(0xffffffffu, c);
+      if (c) {
+        const int pos = C + __popc(ball & below);
+        if (pos < kCandCap) {
+          cand_v[wib][pos] = v[i];
+          cand_j[wib][pos] = j;
+        }
+      }
+      C += __popc(ball);
+    }
+    kept_bits[wib][lane] = 0;
+    __syncwarp();
+    if (C <= kCandCap) {
+      for (int c = lane; c < C; c += 32) {
+        const double sv = cand_v[wib][c];
+        const int sj = cand_j[wib][c];
+        int r = 0;
+        for (int c2 = 0; c2 < C; ++c2) {
+          const double o = cand_v[wib][c2];
+          r += (o > sv || (o == sv && cand_j[wib][c2] < sj)) ? 1 : 0;
+        }
+        if (r < kb) atomicOr(&kept_bits[wib][sj >> 5], 1u << (sj & 31));
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < MAXP; ++i) taken |= ((kept_bits[wib][i] >> lane) & 1u) << i;
+      done = true;
+    }
+  }
+  if (!done) {
+    // k_b rounds of a warp arg-max; only the lane that owned the winner
+    // looks for its next candidate
+    auto local_best = [&](double& best, int& bidx) {
+      best = -INFINITY;
+      bidx = kNone;
+#pragma unroll
+      for (int i = 0; i < MAXP; ++i) {
+        const int j = i * 32 + lane;
+        if (j < nb && !((taken >> i) & 1u) && (bidx == kNone || v[i] > best)) {
+          best = v[i];
+          bidx = j;
+        }
+      }
+    };
     double lb;
     int li;
     local_best(lb, li);
@@ -189,7 +254,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ si
           bidx = oi;
         }
       }
-      // only the lane that owned the winner needs a new candidate
       if (bidx != kNone && (bidx & 31) == lane) {
         taken |= 1u << (bidx >> 5);
         local_best(lb, li);
@@ -197,13 +261,20 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ si
     }
   }
   int pos = 0;
-  for (int i = 0; i < nper; ++i) {
+#pragma unroll
+  for (int i = 0; i < MAXP; ++i) {
     const int j = i * 32 + lane;
     const bool mine = j < nb && ((taken >> i) & 1u);
     const uint32_t ball = __ballot_sync(0xffffffffu, mine);
     if (mine) out[pos + __popc(ball & ((1u << lane) - 1u))] = j;
     pos += __popc(ball);
   }
+}
+
+template <int MAXP>
+static void launch_topk(const double* sigma, int32_t* idx, int rows, int nb, int kb, cudaStream_t cs) {
+  topk_kernel<MAXP><<<(rows + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, cs>>>(sigma, idx, rows,
+                                                                                      nb, kb);
 }
 
 // Scores and top-k from pooled block means (float64 [B, H, nb, d]).
@@ -213,7 +284,13 @@ rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, cons
   const int tiles = (nb + kScTile - 1) / kScTile;
   score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, 0, cs>>>(qbar, kbar, sigma, s->H, s->d, nb);
   const int rows = s->B * s->H * nb;
-  topk_kernel<<<(rows + 7) / 8, 256, 0, cs>>>(sigma, idx, rows, nb, s->k_b);
+  const int nper = (nb + 31) / 32;
+  if (nper <= 4) launch_topk<4>(sigma, idx, rows, nb, s->k_b, cs);
+  else if (nper <= 8) launch_topk<8>(sigma, idx, rows, nb, s->k_b, cs);
+  else if (nper <= 16) launch_topk<16>(sigma, idx, rows, nb, s->k_b, cs);
+  else if (nper <= 20) launch_topk<20>(sigma, idx, rows, nb, s->k_b, cs);
+  else if (nper <= 24) launch_topk<24>(sigma, idx, rows, nb, s->k_b, cs);
+  else launch_topk<kMaxPerLane>(sigma, idx, rows, nb, s->k_b, cs);
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 

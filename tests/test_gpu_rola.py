@@ -65,6 +65,35 @@ def test_select_blocks_bitexact(cfg):
     assert (np.diff(idx_gpu, axis=-1) > 0).all() and idx_gpu.min() >= 0 and idx_gpu.max() < w.n_blocks
 
 
+@pytest.mark.parametrize("T,Hg,W,kb", [
+    (4, 40, 40, 32),   # 100 blocks of 64: largest k_b of the candidate path
+    (4, 40, 40, 33),   # k_b above 32: arg-max rounds
+    (4, 60, 80, 7),    # 300 blocks: more lanes' worth of scores per lane
+])
+def test_select_kb_paths(T, Hg, W, kb):
+    w = synth.Workload("sel", 1, 3, 64, T, Hg, W, 64, 0, kb, 16, seed=5)
+    inp = synth.make_inputs(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx_gpu = rb.select_blocks(rb.Shape.of(w), q, k).cpu().numpy()
+    idx_ref, sig = ro.select_all(inp, w.block, w.k_b)
+    ties, bad = mask_mismatch(idx_gpu, idx_ref, sig, w.k_b)
+    assert not bad, f"mask rows differ outside near-ties: {bad[:5]}"
+
+
+@pytest.mark.parametrize("T,Hg,W,kb", [(4, 40, 40, 5), (4, 60, 80, 5), (4, 60, 80, 40)])
+def test_select_all_scores_equal(T, Hg, W, kb):
+    """q = 0 makes every score 0: ties go to the lower block index, so each
+    row keeps blocks 0 .. k_b - 1 (300 blocks exceed the candidate buffer)."""
+    w = synth.Workload("ties", 1, 2, 64, T, Hg, W, 64, 0, kb, 16, seed=6)
+    inp = synth.make_inputs(w)
+    inp["q"] = np.zeros_like(inp["q"])
+    q, k, v, P, gate = dev_inputs(inp)
+    idx_gpu = rb.select_blocks(rb.Shape.of(w), q, k).cpu().numpy()
+    idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
+    assert np.array_equal(idx_ref, np.broadcast_to(np.arange(kb, dtype=np.int32), idx_ref.shape))
+    assert np.array_equal(idx_gpu, idx_ref)
+
+
 @pytest.mark.parametrize("cfg,heads", [(0, [0, 1]), (1, [0, 11]), (3, [0, 39])])
 def test_block_states(cfg, heads):
     w, inp = workload_inputs(cfg)
