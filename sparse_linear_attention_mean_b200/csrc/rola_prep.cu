@@ -7,16 +7,16 @@
 // means), and a rotary low-rank linear branch restores the dropped context
 // (per-block states S_j = rho^T V, z_j = sum psi, rho = R(t, y, x) phi(K P_h)).
 //
-// Persistent CTAs (256 threads) walk (batch, head, block) items.  Thread 0
-// TMA-loads the q, k and v tiles of the next item (128-byte swizzle) while
-// all warps work on the current one:
-//   * block sums of q and k over the valid tokens in float64 (exact for bf16),
-//     divided by the count;
+// Persistent CTAs (256 threads, two per SM) walk (batch, head, block) items.
+// Thread 0 TMA-loads the item's k and v tiles (128-byte swizzle) while every
+// thread loads its share of the q tile straight into registers; the other
+// CTA on the SM computes meanwhile.  Per item:
+//   * block sums of q and k over the valid tokens in float64 (exact for bf16;
+//     rows past N are zero), divided by the count;
 //   * K P_h with mma.sync, psi = phi(.), rho = rotation by a per-CTA cos/sin
-//     table of the 3-D rotary angles, written as bf16 hi + lo over the (then
-//     dead) q tile;
+//     table of the 3-D rotary angles, written as bf16 hi + lo;
 //   * S_j^T = V^T rho with mma.sync (hi and lo parts), z_j = sum of psi.
-// The kernel is bound by HBM: 96 KB read and ~18 KB written per item.
+// The kernel is bound by HBM: 96 KB read and ~16.5 KB written per item.
 #include <math.h>
 
 #include "rola_common.cuh"
@@ -32,16 +32,19 @@ constexpr int kTabCap = 1024;
 
 template <int R>
 struct Layout {
-  static constexpr uint32_t stage_bytes = 3 * TILE;  // q, k, v
-  static constexpr uint32_t pt_off = 2 * stage_bytes;
+  static constexpr uint32_t stage_bytes = 2 * TILE;  // k, v
   static constexpr int PS = R + 8;                   // padded row of P_h and rho (bf16)
+  static constexpr uint32_t RHO_BYTES = BS * PS * 2;  // one of hi / lo
+  // the pooling partials [8 warps][q, k][128] float64 share this buffer with
+  // rho (written once the partials are consumed)
+  static constexpr uint32_t PART_BYTES = 8 * 2 * D * 8;
+  static constexpr uint32_t rho_off = stage_bytes;
+  static constexpr uint32_t pt_off = rho_off + (2 * RHO_BYTES > PART_BYTES ? 2 * RHO_BYTES : PART_BYTES);
   static constexpr uint32_t misc_off = pt_off + D * PS * 2;
-  static constexpr uint32_t RHO_BYTES = BS * PS * 2;  // one of hi / lo, inside the q tile
-  static_assert(2 * RHO_BYTES <= TILE, "rho must fit in the q tile");
 };
 
 struct Misc {
-  uint64_t full[2];
+  uint64_t full;
   int abort;
   int cur_h;
   float zpart[8][32];
@@ -51,6 +54,7 @@ struct Misc {
 struct Params {
   int B, H, N, nb, Hg, W, items;
   int do_pool;
+  const uint16_t* q;  // [B, N, H, d] bf16 (pooling only)
   double* qbar;  // [B, H, nb, d] float64, or null
   double* kbar;
   const uint16_t* P;
@@ -87,9 +91,9 @@ ROLA_DEV uint32_t sw_off(int row, int col) {
 }
 
 template <int R>
-__global__ void __launch_bounds__(kThreads, 1)
-    rola_prep_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const Params p) {
+__global__ void __launch_bounds__(kThreads, 2)
+    rola_prep_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const Params p) {
   using Ly = Layout<R>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -102,8 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.items > (int)blockIdx.x ? (p.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (tid == 0) {
-    mbar_init(&M.full[0], 1);
-    mbar_init(&M.full[1], 1);
+    mbar_init(&M.full, 1);
     M.abort = 0;
     M.cur_h = -1;
     fence_barrier_init();
@@ -128,35 +131,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue = [&](int it) {
     int b, h, blk;
     decode(it, b, h, blk);
-    const int st = it & 1;
-    uint8_t* base = smem + st * Ly::stage_bytes;
-    mbar_expect_tx(&M.full[st], p.do_pool ? 3 * TILE : 2 * TILE);
+    mbar_expect_tx(&M.full, 2 * TILE);
     for (int ka = 0; ka < 2; ++ka) {
-      if (p.do_pool) tma_load_4d(base + ka * (BS * 128), &tmQ, &M.full[st], ka * 64, h, blk * BS, b);
-      tma_load_4d(base + TILE + ka * (BS * 128), &tmK, &M.full[st], ka * 64, h, blk * BS, b);
-      tma_load_4d(base + 2 * TILE + ka * (BS * 128), &tmV, &M.full[st], ka * 64, h, blk * BS, b);
+      tma_load_4d(smem + ka * (BS * 128), &tmK, &M.full, ka * 64, h, blk * BS, b);
+      tma_load_4d(smem + TILE + ka * (BS * 128), &tmV, &M.full, ka * 64, h, blk * BS, b);
     }
   };
   if (tid == 0 && my_items > 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    issue(0);
   }
+  // pooling: thread = (row group rg of rows rg + 16 i, 8-channel chunk c8)
+  const int rg = tid >> 4, c8 = tid & 15;
+  double* part = reinterpret_cast<double*>(smem + Ly::rho_off);  // [8][2][D]
 
   bool ok = true;
   int it = 0;
   for (; ok && it < my_items; ++it) {
-    const int st = it & 1;
-    // the other stage was released by the __syncthreads closing the last item
-    if (tid == 0 && it + 1 < my_items) issue(it + 1);
+    // the stage was released by the __syncthreads closing the last item
+    if (tid == 0) issue(it);
     int b, h, blk;
     decode(it, b, h, blk);
     const size_t bh = (size_t)b * p.H + h;
     const int tok0 = blk * BS;
     const int valid = min(BS, p.N - tok0);
-    uint8_t* sq = smem + st * Ly::stage_bytes;
-    uint8_t* sk = sq + TILE;
+    uint8_t* sk = smem;
     uint8_t* sv = sk + TILE;
+    uint4 qv[8];
+    if (p.do_pool) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = rg + 16 * i;
+        qv[i] = row < valid ? __ldg(reinterpret_cast<const uint4*>(
+                                  p.q + (((size_t)b * p.N + tok0 + row) * p.H + h) * D + c8 * 8))
+                            : make_uint4(0, 0, 0, 0);
+      }
+    }
     // P_h (rows d, padded) when the head changes
     if (h != M.cur_h) {
       for (int e = tid; e < D * (R / 8); e += kThreads) {
@@ -167,17 +177,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       if (tid == 0) M.cur_h = h;
     }
-    if (!(ok = mbar_wait(&M.full[st], (it >> 1) & 1, abort))) break;
+    if (!(ok = mbar_wait(&M.full, it & 1, abort))) break;
 
-    // ---- block means of q and k (float64: the bf16 sums are exact)
+    // ---- block sums of q and k (float64: the bf16 sums are exact); rows past
+    // N are zero in both (q not loaded, k zero-filled by the copy)
     if (p.do_pool) {
-      const uint8_t* tile = tid < 128 ? sq : sk;
-      const int c = tid & 127;
-      double acc = 0.0;
-      for (int r = 0; r < valid; ++r)
-        acc += (double)bf16_lo(*reinterpret_cast<const uint16_t*>(tile + sw_off(r, c)));
-      double* dst = tid < 128 ? p.qbar : p.kbar;
-      dst[(bh * p.nb + blk) * D + c] = acc / (double)valid;
+      double aq[8], ak[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.0;
+      const uint32_t koff = (uint32_t)((c8 >> 3) * (BS * 128) + rg * 128 + (((c8 & 7) ^ (rg & 7)) << 4));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 kw = *reinterpret_cast<const uint4*>(sk + koff + i * 16 * 128);
+        const uint32_t qa[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+        const uint32_t ka[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          aq[2 * e] += (double)bf16_lo(qa[e]);
+          aq[2 * e + 1] += (double)bf16_hi(qa[e]);
+          ak[2 * e] += (double)bf16_lo(ka[e]);
+          ak[2 * e + 1] += (double)bf16_hi(ka[e]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        aq[e] += __shfl_xor_sync(0xffffffffu, aq[e], 16);
+        ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], 16);
+      }
+      if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          part[(warp * 2 + 0) * D + c8 * 8 + e] = aq[e];
+          part[(warp * 2 + 1) * D + c8 * 8 + e] = ak[e];
+        }
+      }
     }
 
     // ---- kt = K P_h : warp w owns token rows [16w, 16w + 16)
@@ -203,11 +236,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    __syncthreads();  // everyone is done with the q tile (pooling): rho goes there
+    __syncthreads();  // pooling partials complete
+    if (p.do_pool) {
+      const int tile = tid >> 7, c = tid & 127;
+      double acc2 = 0.0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) acc2 += part[(w * 2 + tile) * D + c];
+      double* dst = tile == 0 ? p.qbar : p.kbar;
+      dst[(bh * p.nb + blk) * D + c] = acc2 / (double)valid;
+    }
+    __syncthreads();  // partials consumed: rho goes over them
 
-    // ---- psi, rho (hi / lo bf16 into the q tile), partial z
-    uint16_t* rh = reinterpret_cast<uint16_t*>(sq);
-    uint16_t* rl = reinterpret_cast<uint16_t*>(sq + Ly::RHO_BYTES);
+    // ---- psi, rho (hi / lo bf16), partial z
+    uint16_t* rh = reinterpret_cast<uint16_t*>(smem + Ly::rho_off);
+    uint16_t* rl = reinterpret_cast<uint16_t*>(smem + Ly::rho_off + Ly::RHO_BYTES);
     float zp[NT][2];
 #pragma unroll
     for (int j = 0; j < NT; ++j) zp[j][0] = zp[j][1] = 0.f;
@@ -302,29 +344,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();  // stage st is free for item it + 2
   }
-  // drain: if we stopped early, let the copies in flight land before exiting
-  if (tid == 0) {
+  // drain: if we stopped early, let the copy in flight land before exiting
+  if (tid == 0 && it < my_items) {
     int no_abort = 0;
-    for (int j = it; j < my_items && j <= it + 1; ++j) mbar_wait(&M.full[j & 1], (j >> 1) & 1, &no_abort);
+    mbar_wait(&M.full, it & 1, &no_abort);
   }
   if (tid == 0 && M.abort && p.dev_err) atomicOr(p.dev_err, ROLA_DEVERR_TIMEOUT);
 }
 
 template <int R>
-static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                            Params prm, cudaStream_t cs) {
+static rola_status_t launch(const rola_shape_t* s, const uint16_t* k, const uint16_t* v, Params prm,
+                            cudaStream_t cs) {
   using Ly = Layout<R>;
-  CUtensorMap mq, mk, mv;
-  if (!rola_host::make_act_map(&mk, k, s, BS) || !rola_host::make_act_map(&mv, v, s, BS) ||
-      !rola_host::make_act_map(&mq, q ? q : k, s, BS))
+  CUtensorMap mk, mv;
+  if (!rola_host::make_act_map(&mk, k, s, BS) || !rola_host::make_act_map(&mv, v, s, BS))
     return ROLA_ERR_CUDA;
   const size_t smem = Ly::misc_off + sizeof(Misc) + 1024;
   auto kern = rola_prep_kernel<R>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ROLA_ERR_CUDA;
-  const int nsm = rola_host::sm_count();
-  const int grid = prm.items < nsm ? prm.items : nsm;
-  kern<<<grid, kThreads, smem, cs>>>(mq, mk, mv, prm);
+  const int ctas = 2 * rola_host::sm_count();
+  const int grid = prm.items < ctas ? prm.items : ctas;
+  kern<<<grid, kThreads, smem, cs>>>(mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 
@@ -348,6 +389,7 @@ rola_status_t launch_prep_kernel(const rola_shape_t* s, const uint16_t* q, const
   prm.W = s->W;
   prm.items = s->B * s->H * prm.nb;
   prm.do_pool = (q && qbar && kbar) ? 1 : 0;
+  prm.q = q;
   prm.qbar = qbar;
   prm.kbar = kbar;
   prm.P = P;
@@ -363,8 +405,8 @@ rola_status_t launch_prep_kernel(const rola_shape_t* s, const uint16_t* q, const
   }
   for (int i = 0; i < 17; ++i) prm.tab_first[i] = tl.first[i];
   prm.tab_entries = tl.entries <= prep::kTabCap ? tl.entries : 0;
-  if (s->r == 32) return prep::launch<32>(s, q, k, v, prm, cs);
-  return prep::launch<16>(s, q, k, v, prm, cs);
+  if (s->r == 32) return prep::launch<32>(s, k, v, prm, cs);
+  return prep::launch<16>(s, k, v, prm, cs);
 }
 
 }  // namespace rola
