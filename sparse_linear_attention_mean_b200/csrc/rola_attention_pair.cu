@@ -243,15 +243,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 128; ++c)
               if (c >= valid) x[c] = __float_as_uint(-INFINITY);
           }
-          float m0 = -INFINITY, m1 = -INFINITY;
+          // row max in four independent chains (short dependency latency)
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 128; c += 4) {
+          for (int c = 0; c < 128; c += 8) {
             m0 = fmax3(m0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
             m1 = fmax3(m1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+            m2 = fmax3(m2, __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+            m3 = fmax3(m3, __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
           }
           // lazy rescaling: the exponent base m moves only when the row max
           // exceeds it by more than 2^8 (P then stays <= 256)
-          const float mc = fmaxf(m0, m1) * p.scale_log2;
+          const float mc = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * p.scale_log2;
           float alpha = 1.f;
           bool need = false;
           if (first) {
@@ -648,6 +651,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; ok && j < U.nu; ++j) {
           const uint32_t gk = g, gv = g + 1;
           g += 2;
+          // slot 0's pending P.V needs no new tile: it goes out before the
+          // wait for K, which frees its V slot for the copies sooner
+          if (pend_v[0] >= 0 && !(ok = issue_pv(0))) break;
           if (!(ok = mbar_wait(&M.ring_full[gk % NR], (gk / NR) & 1, abort))) break;
           const int mk = U.umask[j];
           users[gv % NR] = __popc(mk);
