@@ -103,6 +103,18 @@ rola_status_t rola_select_blocks(const rola_shape_t* shape, const uint16_t* q, c
                                  int32_t* idx, double* scores_opt, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* The selector above without a caller workspace: its scratch is a fixed
+ * 16 MiB device array inside this library (the pages describe no such call;
+ * it exists for callers that cannot provide device memory at the call site).
+ * Same inputs, output and results as rola_select_blocks (no scores output).
+ * ROLA_ERR_WORKSPACE when rola_select_workspace_bytes(shape) exceeds 16 MiB.
+ * The first call on a device looks up the array's address (set-up work: make
+ * it before any stream capture).  Nothing is allocated and nothing needs
+ * clearing; calls that overlap in time on one device share the array and
+ * race, so callers serialise them. */
+rola_status_t rola_select_blocks_noalloc(const rola_shape_t* shape, const uint16_t* q,
+                                         const uint16_t* k, int32_t* idx, void* stream);
+
 /* ---------------------------------------------------------------- states */
 
 /* Linear-branch key/value states (write-up section 05: the low-rank linear

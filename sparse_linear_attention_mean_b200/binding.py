@@ -22,7 +22,8 @@ DEVERR_TIMEOUT = 0x2
 
 EXPORTS = [
     "rola_status_string", "rola_num_blocks", "rola_kb_from_sparsity",
-    "rola_select_workspace_bytes", "rola_select_blocks", "rola_block_states",
+    "rola_select_workspace_bytes", "rola_select_blocks", "rola_select_blocks_noalloc",
+    "rola_block_states",
     "rola_attention_fwd", "rola_layer_workspace_bytes", "rola_layer_fwd", "rola_layer_fwd_timed",
     "rola_layer_kernel_launches",
     "rola_layer_host_workspace_bytes", "rola_layer_fwd_host",
@@ -95,6 +96,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, nm).argtypes = [sp]
         L.rola_select_blocks.restype = ctypes.c_int
         L.rola_select_blocks.argtypes = [sp, vp, vp, vp, vp, vp, sz, vp]
+        L.rola_select_blocks_noalloc.restype = ctypes.c_int
+        L.rola_select_blocks_noalloc.argtypes = [sp, vp, vp, vp, vp]
         L.rola_block_states.restype = ctypes.c_int
         L.rola_block_states.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rola_attention_fwd.restype = ctypes.c_int

@@ -10,6 +10,8 @@
 #include <float.h>
 #include <math.h>
 
+#include <mutex>
+
 #include "rola_common.cuh"
 #include "rola_internal.h"
 
@@ -327,6 +329,65 @@ extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_
       rola_internal::round_up(2 * (size_t)s->B * s->H * nb * s->d * sizeof(double), 256));
   if (scores_opt) sig = scores_opt;
 
+  pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
+  if (cudaGetLastError() != cudaSuccess) return ROLA_ERR_CUDA;
+  return select_from_pooled(s, qbar, kbar, sig, idx, cs);
+}
+
+// ---------------------------------------------------------------- selector without a workspace
+// The same selector (pooling, scores, top-k: the kernels above) with its
+// scratch in a fixed device array of this library instead of a caller
+// workspace.  It serves callers that cannot hand over device memory at the
+// call site: a host-side plugin or language binding that holds only the q, k
+// and idx buffers and has no device allocator of its own.  Nothing is
+// allocated per call: the array exists once per device for the life of the
+// context, and its address is looked up (cudaGetSymbolAddress) on the first
+// call on each device -- so that first call does set-up work and should come
+// before any stream capture.  Every scratch word is written before it is
+// read, so nothing needs clearing between calls; calls that overlap in time
+// on one device (several streams or host threads) share the array and race.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device, or null.
+void* scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
+    g_scratch_addr[dev] = p;
+  }
+  return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" rola_status_t rola_select_blocks_noalloc(const rola_shape_t* s, const uint16_t* q,
+                                                    const uint16_t* k, int32_t* idx, void* stream) {
+  rola_status_t st = rola_internal::check_shape(s);
+  if (st != ROLA_OK) return st;
+  if (!q || !k || !idx) return ROLA_ERR_INVALID_ARG;
+  if (!rola_host::aligned(q, 16) || !rola_host::aligned(k, 16) || !rola_host::aligned(idx, 4))
+    return ROLA_ERR_ALIGNMENT;
+  const int nb = rola_num_blocks(s);
+  if (nb > 32 * kMaxPerLane) return ROLA_ERR_UNSUPPORTED;
+  // the scratch this shape needs must fit the fixed array
+  if (rola_select_workspace_bytes(s) > kNoAllocScratchBytes) return ROLA_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(scratch_on_current_device());
+  if (!ws) return ROLA_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  double* qbar = reinterpret_cast<double*>(ws);
+  double* kbar = qbar + (size_t)s->B * s->H * nb * s->d;
+  double* sig = reinterpret_cast<double*>(
+      ws + rola_internal::round_up(2 * (size_t)s->B * s->H * nb * s->d * sizeof(double), 256));
   pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
   if (cudaGetLastError() != cudaSuccess) return ROLA_ERR_CUDA;
   return select_from_pooled(s, qbar, kbar, sig, idx, cs);
