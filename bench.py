@@ -144,7 +144,9 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(w, inp) -> dict:
-    dt, flop, text = oracle_sample(w, inp, heads=(0,), qblocks=range(0, w.n_blocks, 4))
+    # about 10 s of host work: every query block of four heads
+    heads = tuple(sorted({0, w.H // 3, (2 * w.H) // 3, w.H - 1}))
+    dt, flop, text = oracle_sample(w, inp, heads=heads, qblocks=range(w.n_blocks))
     return {"value": flop / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": text + f"; {dt:.1f} s"}
 
@@ -158,7 +160,7 @@ def run_reference(args) -> int:
     from sparse_linear_attention_mean_b200 import synth
     w = synth.WORKLOADS[WORKLOAD_ID]
     inp = synth.make_inputs(w)
-    qblocks = range(0, w.n_blocks, 8)     # bounded sample per step: 74 query blocks of one head
+    qblocks = range(w.n_blocks)           # bounded sample per step: every query block of one head
     for _ in range(args.warmup):
         oracle_sample(w, inp, heads=(0,), qblocks=qblocks)
     times, flop, text = [], 0.0, ""
@@ -369,6 +371,9 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projection timing")
+    ap.add_argument("--fp8-only", action="store_true",
+                    help="time only the FP8 projection (x [rows, 5120] -> [rows, 5120]); profiling captures")
+    ap.add_argument("--fp8-rows", type=int, default=75600, help="rows of x for --fp8-only")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (per-head work unchanged; for profiling captures)")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
@@ -376,6 +381,10 @@ def main() -> int:
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.fp8_only:
+        import torch
+        print(json.dumps({"fp8_projection": fp8_projection(args.fp8_rows, 5120, torch.cuda.current_stream())}))
+        return 0
     return run_gpu(args)
 
 
