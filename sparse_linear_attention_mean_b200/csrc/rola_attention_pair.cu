@@ -98,6 +98,7 @@ struct Misc {
   int err;
   float zU[2][32];
   float2 tab[kTabCap];  // (cos, sin) of pos * freq per rotation pair and grid position
+  int4 rope_pair[16];   // per rotation pair: table base, stride per position, axis
   UnitList L[2];
 };
 
@@ -191,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   // rotary cos/sin table, once per (persistent) CTA
+  if (tid < R / 2) M.rope_pair[tid] = make_int4(p.tab_base[tid], p.tab_stride[tid], p.rope.axis[tid], 0);
   for (int e = tid; e < p.tab_entries; e += kThreads) {
     int pr = 0;
     while (pr + 1 < R / 2 && e >= p.tab_first[pr + 1]) ++pr;
@@ -288,8 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           first = false;
           if (__any_sync(0xffffffffu, need)) {
             // O holds the previous P.V, complete because that MMA was issued
-            // before this S; the next P.V waits for p_full.
-#pragma unroll
+            // before this S; the next P.V waits for p_full.  (Rare: rolled.)
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
               uint32_t o[32];
               tmem_ld32(oc + c * 32, o);
@@ -309,48 +311,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         // so that the epilogue is out = O / l.  rho'_q (bf16 hi + lo) goes to
         // columns [32, 32 + r) of this slot's S buffer as the A operand of
         // that MMA; q P_h sits in columns [0, r).
+        // This code runs once per unit, cold in the instruction cache, so it
+        // is written as short rolled loops over 8-column chunks.
         if (!(ok = warp_wait(&M.qt_full[s], uc & 1, abort))) break;
         tc_fence_after();
-        uint32_t qt[32];
-        if constexpr (R == 32) {
-          tmem_ld32(sc, qt);
-        } else {
-          tmem_ld16(sc, *reinterpret_cast<uint32_t(*)[16]>(&qt[0]));
-        }
-        tmem_wait_ld();
         const int n = U.a[s] * BM + row;
         const int nn = n < p.N ? n : p.N - 1;
-        const int pt_ = nn / (p.Hg * p.W), py = (nn / p.W) % p.Hg, px = nn % p.W;
-        float2 cs[R / 2];
-#pragma unroll
-        for (int pr = 0; pr < R / 2; ++pr) {
-          const int ax = p.rope.axis[pr];
-          cs[pr] = M.tab[p.tab_base[pr] + (ax == 0 ? pt_ : (ax == 1 ? py : px)) * p.tab_stride[pr]];
-        }
-#pragma unroll
-        for (int c = 0; c < R; ++c) qt[c] = __float_as_uint(phi(__uint_as_float(qt[c])));  // psi_q
+        const int hw = p.Hg * p.W;
+        const int pt_ = nn / hw, rem = nn - pt_ * hw;
+        const int py = rem / p.W, px = rem - py * p.W;
         if (!(ok = warp_wait(&M.zu_ready[s], uc & 1, abort))) break;
+        // pass 1: den = psi_q . z_U
         float den = 0.f;
+#pragma unroll 1
+        for (int c8 = 0; c8 < R / 8; ++c8) {
+          uint32_t v[8];
+          tmem_ld8(sc + c8 * 8, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < R; ++c) den = fmaf(__uint_as_float(qt[c]), M.zU[s][c], den);
+          for (int e = 0; e < 8; ++e) den = fmaf(phi_fast(__uint_as_float(v[e])), M.zU[s][c8 * 8 + e], den);
+        }
         const bool have_o = U.cnt[s] > 0;
         const float lsum = have_o ? l : 1.f;
         const float scale = U.lin_empty[s] ? 0.f : p.gate[U.h] * lsum / den;
-        uint32_t rh[R / 2], rl[R / 2];
+        // pass 2: rho'_q = R(t, y, x) psi_q * scale as bf16 hi + lo
+#pragma unroll 1
+        for (int c8 = 0; c8 < R / 8; ++c8) {
+          uint32_t v[8], rh[4], rl[4];
+          tmem_ld8(sc + c8 * 8, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int pr = 0; pr < R / 2; ++pr) {
-          const float x0 = __uint_as_float(qt[2 * pr]), x1 = __uint_as_float(qt[2 * pr + 1]);
-          const float r0 = (x0 * cs[pr].x - x1 * cs[pr].y) * scale;
-          const float r1 = (x0 * cs[pr].y + x1 * cs[pr].x) * scale;
-          rh[pr] = pack_bf16(r0, r1);
-          rl[pr] = pack_bf16(r0 - bf16_lo(rh[pr]), r1 - bf16_hi(rh[pr]));
-        }
-        if constexpr (R == 32) {
-          tmem_st16(sc + 32, rh);
-          tmem_st16(sc + 48, rl);
-        } else {
-          tmem_st8(sc + 32, rh);
-          tmem_st8(sc + 40, rl);
+          for (int i = 0; i < 4; ++i) {
+            const int4 rp = M.rope_pair[c8 * 4 + i];
+            const float2 c = M.tab[rp.x + (rp.z == 0 ? pt_ : (rp.z == 1 ? py : px)) * rp.y];
+            const float x0 = phi_fast(__uint_as_float(v[2 * i])), x1 = phi_fast(__uint_as_float(v[2 * i + 1]));
+            const float r0 = (x0 * c.x - x1 * c.y) * scale;
+            const float r1 = (x0 * c.y + x1 * c.x) * scale;
+            rh[i] = pack_bf16(r0, r1);
+            rl[i] = pack_bf16(r0 - bf16_lo(rh[i]), r1 - bf16_hi(rh[i]));
+          }
+          tmem_st4(sc + 32 + c8 * 4, rh);
+          tmem_st4(sc + 32 + R / 2 + c8 * 4, rl);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -360,21 +361,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const float inv_l = 1.f / lsum;
         const bool write = n < p.N;
-        uint16_t* orow = p.out + (((size_t)U.b * p.N + (write ? n : 0)) * p.H + U.h) * D;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t o[64];
-          tmem_ld32_at<0>(oc + hf * 64, o);
-          tmem_ld32_at<32>(oc + hf * 64 + 32, o);
+        uint4* orow = reinterpret_cast<uint4*>(p.out + (((size_t)U.b * p.N + (write ? n : 0)) * p.H + U.h) * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t o[16];
+          tmem_ld16(oc + c * 16, o);
           tmem_wait_ld();
-          uint32_t wv[32];
+          uint32_t wv[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
+          for (int e = 0; e < 8; ++e)
             wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
           if (write) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + hf * 64);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+            orow[2 * c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            orow[2 * c + 1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
           }
         }
         tc_fence_before();
@@ -674,18 +673,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (ok) mma_commit(&M.ring_empty[gk % NR]);
         }
-#pragma unroll
-        for (int s = 0; s < 2; ++s)
-          if (ok && pend_v[s] >= 0) ok = issue_pv(s);
-        if (!ok) break;
-        // tile end: q P_h into the (now free) S columns; Q is then free for
-        // the next unit.  Then O += rho'_q S_U with rho'_q read from tensor
-        // memory (written by the softmax warps) and S_U from the gather.
+        // tile end, per slot as soon as its last P.V is out: q P_h into the
+        // (now free) S columns; Q is then free for the next unit.  Then
+        // O += rho'_q S_U with rho'_q read from tensor memory (written by the
+        // softmax warps) and S_U from the gather.
         if (!(ok = mbar_wait(&M.pt_full, u & 1, abort))) break;
-        tc_fence_after();
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
-          if (!U.active[s]) continue;
+          if (ok && pend_v[s] >= 0) ok = issue_pv(s);
+          if (!ok || !U.active[s]) continue;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tm + s_col(s), dq0[s] + kstep_k_sw128(BM, kk), desc_k_sw128(sPT, 32, kk), idesc_qt,
@@ -693,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&M.qt_full[s]);
           mma_commit(&M.q_empty[s]);
         }
+        if (!ok) break;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           if (!ok || !U.active[s]) continue;

@@ -220,6 +220,12 @@ ROLA_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+ROLA_DEV void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
+}
 ROLA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -277,6 +283,11 @@ ROLA_DEV void tmem_st32_at(uint32_t taddr, const uint32_t (&r)[N]) {
       : "memory");
 }
 
+ROLA_DEV void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
 ROLA_DEV void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
                    taddr),
@@ -313,6 +324,9 @@ ROLA_DEV void rope_sincos(int pos, double freq, float* s, float* c) {
 
 // phi(u) = elu(u) + 1.
 ROLA_DEV float phi(float u) { return u > 0.f ? u + 1.f : expf(u); }
+// The same with the fast exponential intrinsic (a few ulp; short code for
+// paths that run cold in the instruction cache).
+ROLA_DEV float phi_fast(float u) { return u > 0.f ? u + 1.f : __expf(u); }
 
 // ---------------------------------------------------------------- packed fp32
 
