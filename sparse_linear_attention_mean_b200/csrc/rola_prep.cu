@@ -63,7 +63,7 @@ struct Params {
   int32_t* dev_err;
   RopeTable rope;
   int tab_base[16], tab_stride[16], tab_first[17];
-  int tab_entries;  // 0: table too large, sin/cos computed directly
+  int tab_entries;  // cos/sin table entries (the table always fits: see prep_kernel_supports)
 };
 
 ROLA_DEV void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
@@ -89,6 +89,19 @@ ROLA_DEV uint32_t sw_off(int row, int col) {
   return (uint32_t)((col >> 6) * (BS * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
                     (col & 7) * 2);
 }
+
+// bf16 -> float64 times 2^-896, exactly: the bf16 sign, exponent and
+// mantissa bits go to their places in the high word of a float64, whose
+// exponent bias is 1023 instead of 127 (denormals map to denormals).  This
+// keeps the conversion on the integer pipe; the block sums are multiplied by
+// 2^896 at the end, which is exact.
+ROLA_DEV double bf16lo_f64s(uint32_t w) {
+  return __hiloint2double((int)(((w << 16) & 0x80000000u) | ((w << 13) & 0x0fffe000u)), 0);
+}
+ROLA_DEV double bf16hi_f64s(uint32_t w) {
+  return __hiloint2double((int)((w & 0x80000000u) | ((w >> 3) & 0x0fffe000u)), 0);
+}
+constexpr double kTwo896 = 0x1p896;
 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -179,8 +192,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (!(ok = mbar_wait(&M.full, it & 1, abort))) break;
 
-    // ---- block sums of q and k (float64: the bf16 sums are exact); rows past
-    // N are zero in both (q not loaded, k zero-filled by the copy)
+    // ---- block sums of q and k (float64, scaled by 2^-896: the bf16 sums are
+    // exact); rows past N are zero in both (q not loaded, k zero-filled by
+    // the copy)
     if (p.do_pool) {
       double aq[8], ak[8];
 #pragma unroll
@@ -193,10 +207,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t ka[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          aq[2 * e] += (double)bf16_lo(qa[e]);
-          aq[2 * e + 1] += (double)bf16_hi(qa[e]);
-          ak[2 * e] += (double)bf16_lo(ka[e]);
-          ak[2 * e + 1] += (double)bf16_hi(ka[e]);
+          aq[2 * e] += bf16lo_f64s(qa[e]);
+          aq[2 * e + 1] += bf16hi_f64s(qa[e]);
+          ak[2 * e] += bf16lo_f64s(ka[e]);
+          ak[2 * e + 1] += bf16hi_f64s(ka[e]);
         }
       }
 #pragma unroll
@@ -243,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int w = 0; w < 8; ++w) acc2 += part[(w * 2 + tile) * D + c];
       double* dst = tile == 0 ? p.qbar : p.kbar;
-      dst[(bh * p.nb + blk) * D + c] = acc2 / (double)valid;
+      dst[(bh * p.nb + blk) * D + c] = (acc2 * kTwo896) / (double)valid;
     }
     __syncthreads();  // partials consumed: rho goes over them
 
@@ -263,20 +277,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int nj = 0; nj < NT; ++nj) {
         const int col = nj * 8 + 2 * t4;
         const int pr = col >> 1;
-        const float p0 = vok ? phi(acc[nj][2 * half]) : 0.f;
-        const float p1 = vok ? phi(acc[nj][2 * half + 1]) : 0.f;
+        const float p0 = vok ? phi_fast(acc[nj][2 * half]) : 0.f;
+        const float p1 = vok ? phi_fast(acc[nj][2 * half + 1]) : 0.f;
         zp[nj][0] += p0;
         zp[nj][1] += p1;
         const int ax = p.rope.axis[pr];
         const int pos = ax == 0 ? pt : (ax == 1 ? py : px);
-        float sn, cs;
-        if (p.tab_entries) {
-          const float2 v = M.tab[p.tab_base[pr] + pos * p.tab_stride[pr]];
-          cs = v.x;
-          sn = v.y;
-        } else {
-          rope_sincos(pos, p.rope.freq[pr], &sn, &cs);
-        }
+        const float2 v = M.tab[p.tab_base[pr] + pos * p.tab_stride[pr]];
+        const float cs = v.x, sn = v.y;
         const float r0 = p0 * cs - p1 * sn, r1 = p0 * sn + p1 * cs;
         const uint32_t hi = pack_bf16(r0, r1);
         const uint32_t lo = pack_bf16(r0 - bf16_lo(hi), r1 - bf16_hi(hi));
@@ -371,8 +379,14 @@ static rola_status_t launch(const rola_shape_t* s, const uint16_t* k, const uint
 
 }  // namespace prep
 
+// d = 128, 128-token blocks and a latent grid whose rotary table fits in
+// shared memory (other shapes take the per-block state kernel and the
+// separate pooling pass).
 bool prep_kernel_supports(const rola_shape_t* s) {
-  return s->d == 128 && s->block == 128 && (s->r == 16 || s->r == 32);
+  if (!(s->d == 128 && s->block == 128 && (s->r == 16 || s->r == 32))) return false;
+  const int rh = 2 * (s->r / 6), rt = s->r - 2 * rh;
+  const long long entries = (long long)s->T * (rt / 2) + (long long)(s->Hg + s->W) * (rh / 2);
+  return entries <= prep::kTabCap;
 }
 
 // Block means (if q, qbar and kbar are given) and block states of every
@@ -404,7 +418,8 @@ rola_status_t launch_prep_kernel(const rola_shape_t* s, const uint16_t* q, const
     prm.tab_stride[i] = tl.stride[i];
   }
   for (int i = 0; i < 17; ++i) prm.tab_first[i] = tl.first[i];
-  prm.tab_entries = tl.entries <= prep::kTabCap ? tl.entries : 0;
+  if (tl.entries > prep::kTabCap) return ROLA_ERR_UNSUPPORTED;
+  prm.tab_entries = tl.entries;
   if (s->r == 32) return prep::launch<32>(s, k, v, prm, cs);
   return prep::launch<16>(s, k, v, prm, cs);
 }

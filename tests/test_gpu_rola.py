@@ -223,7 +223,7 @@ def test_bad_index_reported_not_trapped():
         check_close(o[0, lo:hi, 0, :], rows)
 
 
-@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("cfg", [0, 1, 3])
 def test_layer_entry_points(cfg):
     w, inp = workload_inputs(cfg)
     shape = rb.Shape.of(w)
