@@ -73,21 +73,23 @@ struct Layout {
   static constexpr uint32_t P_OFF = 0;  // bf16 P over the first 64 columns of its S buffer
 };
 
+constexpr int NL = 3;        // unit lists in flight: the producer builds one unit ahead
+constexpr int kMaxBlocks = 1024;  // n_blocks limit (the list merge keeps one bit per block)
+
 struct UnitList {
   int b, h, a[2];
   int active[2];
   int nu;
   int cnt[2];
   int lin_empty[2];
-  int raw[2][kMaxKept];
-  int ulist[kMaxUnion];
+  uint16_t ulist[kMaxUnion];
   uint8_t umask[kMaxUnion];
 };
 
 constexpr int kTabCap = 1024;  // cos/sin entries of the rotary table in shared memory
 
 struct Misc {
-  uint64_t list_full[2], list_empty[2];
+  uint64_t list_full[NL], list_empty[NL];
   uint64_t q_full[2], q_empty[2];
   uint64_t ring_full[NR], ring_empty[NR];
   uint64_t s_full[2], p_full[2];
@@ -99,7 +101,8 @@ struct Misc {
   float zU[2][32];
   float2 tab[kTabCap];  // (cos, sin) of pos * freq per rotation pair and grid position
   int4 rope_pair[16];   // per rotation pair: table base, stride per position, axis
-  UnitList L[2];
+  uint32_t kept_bits[2][kMaxBlocks / 32];  // list merge scratch of the producer
+  UnitList L[NL];
 };
 
 struct Params {
@@ -113,6 +116,7 @@ struct Params {
   const float* z_glb;
   const float* gate;
   uint16_t* out;
+  int out_32b;  // out is 32-byte aligned: the epilogue stores 32 bytes at a time
   int32_t* dev_err;
   RopeTable rope;
   // rotary table: entry of pair pr at position pos = tab_base[pr] + pos * tab_stride[pr];
@@ -163,9 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.dev_err && (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)) return;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NL; ++i) {
       mbar_init(&M.list_full[i], 1);
       mbar_init(&M.list_empty[i], 1 + 2 * 128 + 64);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&M.q_full[i], 1);
       mbar_init(&M.q_empty[i], 1);
       mbar_init(&M.s_full[i], 1);
@@ -220,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t nsc = 0, uc = 0;
     bool ok = true;
     for (int u = 0; ok && u < my_units; ++u) {
-      const int buf = u & 1;
-      if (!(ok = warp_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+      const int buf = u % NL;
+      if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
       const UnitList& U = M.L[buf];
       if (U.active[s]) {
         float m = 0.f, l = 0.f;
@@ -372,8 +378,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 8; ++e)
             wv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
           if (write) {
-            orow[2 * c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            orow[2 * c + 1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+            if (p.out_32b) {
+              // one 32-byte store (rows start 256-byte apart from a 32-byte aligned base)
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(orow + 2 * c),
+                           "r"(wv[0]), "r"(wv[1]), "r"(wv[2]), "r"(wv[3]), "r"(wv[4]), "r"(wv[5]),
+                           "r"(wv[6]), "r"(wv[7])
+                           : "memory");
+            } else {
+              orow[2 * c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+              orow[2 * c + 1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+            }
           }
         }
         tc_fence_before();
@@ -396,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t uc[2] = {0, 0};
       bool ok = true;
       for (int u = 0; ok && u < my_units; ++u) {
-        const int buf = u & 1;
-        if (!(ok = warp_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+        const int buf = u % NL;
+        if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
         const UnitList& U = M.L[buf];
         const int b = U.b, h = U.h;
         const size_t bh = (size_t)b * p.H + h;
@@ -499,93 +513,114 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
       }
-      for (int u = 0; ok && u < my_units; ++u) {
-        const int buf = u & 1;
-        if (u >= 2 && !(ok = warp_wait(&M.list_empty[buf], ((u >> 1) - 1) & 1, abort))) break;
+      // Unit list of unit u into buffer u % NL, by the whole warp: both kept
+      // lists are validated (in range, above the previous entry of the row;
+      // a bad entry is skipped and reported), marked in one bitmap per slot
+      // and read back as one ascending union with a per-slot mask.
+      auto build_list = [&](int u) -> bool {
+        const int buf = u % NL;
+        if (u >= NL && !warp_wait(&M.list_empty[buf], ((u / NL) - 1) & 1, abort)) return false;
         UnitList& U = M.L[buf];
         int b, h, pair;
         decode_unit(p, (int)blockIdx.x + u * (int)gridDim.x, b, h, pair);
         const int a0 = 2 * pair, a1 = 2 * pair + 1;
         const size_t bh = (size_t)b * p.H + h;
+        M.kept_bits[0][lane] = 0u;
+        M.kept_bits[1][lane] = 0u;
+        __syncwarp();
+        int err = 0;
         for (int i = lane; i < 2 * p.kb; i += 32) {
-          const int s = i / p.kb, a = s ? a1 : a0;
-          U.raw[s][i % p.kb] = a < p.nb ? p.idx[(bh * p.nb + a) * p.kb + i % p.kb] : -1;
+          const int sl = i >= p.kb ? 1 : 0, e = i - sl * p.kb, a = sl ? a1 : a0;
+          if (a >= p.nb) continue;
+          const int32_t* row = p.idx + (bh * p.nb + a) * p.kb;
+          const int v = row[e];
+          if (v >= 0 && v < p.nb && (e == 0 || v > row[e - 1]))
+            atomicOr(&M.kept_bits[sl][v >> 5], 1u << (v & 31));
+          else
+            err = 1;
         }
         __syncwarp();
+        const uint32_t m0 = M.kept_bits[0][lane], m1 = M.kept_bits[1][lane], mu = m0 | m1;
+        int pre = __popc(mu);  // inclusive prefix over lanes: lane w holds blocks [32 w, 32 w + 32)
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, pre, off);
+          if (lane >= off) pre += t;
+        }
+        int pos = pre - __popc(mu);
+        for (uint32_t rem = mu; rem; rem &= rem - 1) {
+          const int bit = __ffs(rem) - 1;
+          U.ulist[pos] = (uint16_t)(lane * 32 + bit);
+          U.umask[pos] = (uint8_t)(((m0 >> bit) & 1u) | (((m1 >> bit) & 1u) << 1));
+          ++pos;
+        }
+        int c0 = __popc(m0), c1 = __popc(m1);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          c0 += __shfl_xor_sync(0xffffffffu, c0, off);
+          c1 += __shfl_xor_sync(0xffffffffu, c1, off);
+        }
+        const int nu = __shfl_sync(0xffffffffu, pre, 31);
+        if (__any_sync(0xffffffffu, err) && lane == 0) M.err = 1;
         if (lane == 0) {
-          // Validate both kept lists (in range, strictly ascending; a bad
-          // entry is skipped and reported) and merge them into one ascending
-          // union with a per-slot membership mask.
           U.b = b;
           U.h = h;
           U.a[0] = a0;
           U.a[1] = a1;
           U.active[0] = a0 < p.nb;
           U.active[1] = a1 < p.nb;
-          int pos[2] = {0, 0}, prev[2] = {-1, -1}, len[2];
-          len[0] = U.active[0] ? p.kb : 0;
-          len[1] = U.active[1] ? p.kb : 0;
-          U.cnt[0] = U.cnt[1] = 0;
-          int nu = 0, err = 0;
-          while (true) {
-            int best = 0x7fffffff;
-            for (int s = 0; s < 2; ++s) {
-              while (pos[s] < len[s]) {
-                const int v = U.raw[s][pos[s]];
-                if (v < 0 || v >= p.nb || v <= prev[s]) { err = 1; ++pos[s]; continue; }
-                break;
-              }
-              if (pos[s] < len[s]) best = min(best, U.raw[s][pos[s]]);
-            }
-            if (best == 0x7fffffff) break;
-            uint8_t mk = 0;
-            for (int s = 0; s < 2; ++s)
-              if (pos[s] < len[s] && U.raw[s][pos[s]] == best) {
-                mk |= (uint8_t)(1u << s);
-                prev[s] = best;
-                ++pos[s];
-                ++U.cnt[s];
-              }
-            U.ulist[nu] = best;
-            U.umask[nu] = mk;
-            ++nu;
-          }
           U.nu = nu;
-          U.lin_empty[0] = U.cnt[0] >= p.nb;
-          U.lin_empty[1] = U.cnt[1] >= p.nb;
-          if (err) M.err = 1;
-          mbar_arrive(&M.list_full[buf]);
-          // K and V of every union entry, gathered by block index; the Q
-          // tiles go out after the first entry so that its K/V load overlaps
-          // the previous unit's tail.
-          auto load_kv = [&](int j) -> bool {
-            const int blk = U.ulist[j];
-            for (int kv = 0; kv < 2; ++kv) {
-              const int slot = g % NR;
-              if (g >= (uint32_t)NR && !mbar_wait(&M.ring_empty[slot], ((g / NR) - 1) & 1, abort)) return false;
-              mbar_expect_tx(&M.ring_full[slot], TILE);
-              const CUtensorMap* mp = kv ? &tmV : &tmK;
-              for (int ka = 0; ka < 2; ++ka)
-                tma_load_4d(smem + Ly::ring_off + slot * TILE + ka * (BN * 128), mp, &M.ring_full[slot],
-                            ka * 64, h, blk * BN, b);
-              ring_par[slot] = (g / NR) & 1;
-              ++g;
-            }
-            return true;
-          };
-          if (nu > 0) ok = load_kv(0);
-          for (int s = 0; s < 2 && ok; ++s) {
-            if (!U.active[s]) continue;
-            if (uc[s] >= 1 && !(ok = mbar_wait(&M.q_empty[s], (uc[s] - 1) & 1, abort))) break;
-            mbar_expect_tx(&M.q_full[s], TILE);
-            for (int ka = 0; ka < 2; ++ka)
-              tma_load_4d(smem + Ly::q_off + s * TILE + ka * (BM * 128), &tmQ, &M.q_full[s], ka * 64, h,
-                          U.a[s] * BM, b);
-            q_par[s] = uc[s] & 1;
-            ++uc[s];
-          }
-          for (int j = 1; ok && j < nu; ++j) ok = load_kv(j);
+          U.cnt[0] = c0;
+          U.cnt[1] = c1;
+          U.lin_empty[0] = c0 >= p.nb;
+          U.lin_empty[1] = c1 >= p.nb;
         }
+        __syncwarp();
+        __threadfence_block();
+        if (lane == 0) mbar_arrive(&M.list_full[buf]);
+        return true;
+      };
+      if (my_units > 0) ok = build_list(0);
+      for (int u = 0; ok && u < my_units; ++u) {
+        const UnitList& U = M.L[u % NL];
+        const int nu = U.nu, b = U.b, h = U.h;
+        // K and V of every union entry, gathered by block index
+        auto load_kv = [&](int j) -> bool {
+          const int blk = U.ulist[j];
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = g % NR;
+            if (g >= (uint32_t)NR && !mbar_wait(&M.ring_empty[slot], ((g / NR) - 1) & 1, abort)) return false;
+            mbar_expect_tx(&M.ring_full[slot], TILE);
+            const CUtensorMap* mp = kv ? &tmV : &tmK;
+            for (int ka = 0; ka < 2; ++ka)
+              tma_load_4d(smem + Ly::ring_off + slot * TILE + ka * (BN * 128), mp, &M.ring_full[slot],
+                          ka * 64, h, blk * BN, b);
+            ring_par[slot] = (g / NR) & 1;
+            ++g;
+          }
+          return true;
+        };
+        // the first entry, then the Q tiles (after the previous unit's last
+        // S MMA has read them), so that the first copy overlaps the previous
+        // unit's tail
+        if (lane == 0) {
+          if (nu > 0) ok = load_kv(0);
+          for (int sl = 0; sl < 2 && ok; ++sl) {
+            if (!U.active[sl]) continue;
+            if (uc[sl] >= 1 && !(ok = mbar_wait(&M.q_empty[sl], (uc[sl] - 1) & 1, abort))) break;
+            mbar_expect_tx(&M.q_full[sl], TILE);
+            for (int ka = 0; ka < 2; ++ka)
+              tma_load_4d(smem + Ly::q_off + sl * TILE + ka * (BM * 128), &tmQ, &M.q_full[sl], ka * 64, h,
+                          U.a[sl] * BM, b);
+            q_par[sl] = uc[sl] & 1;
+            ++uc[sl];
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        // the next unit's list while this unit's copies are in flight
+        if (ok && u + 1 < my_units) ok = build_list(u + 1);
+        if (lane == 0)
+          for (int j = 1; ok && j < nu; ++j) ok = load_kv(j);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         __syncwarp();
       }
@@ -619,8 +654,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < NR; ++i) users[i] = 0;
       bool ok = true;
       for (int u = 0; ok && u < my_units; ++u) {
-        const int buf = u & 1;
-        if (!(ok = mbar_wait(&M.list_full[buf], (u >> 1) & 1, abort))) break;
+        const int buf = u % NL;
+        if (!(ok = mbar_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
         const UnitList& U = M.L[buf];
 #pragma unroll
         for (int s = 0; s < 2; ++s)
@@ -756,6 +791,7 @@ static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint
 bool pair_kernel_supports(const rola_shape_t* s) {
   if (!(s->d == 128 && s->block == 128 && s->k_b <= pairk::kMaxKept && (s->r == 16 || s->r == 32)))
     return false;
+  if (rola_num_blocks(s) > pairk::kMaxBlocks) return false;
   const int rh = 2 * (s->r / 6), rt = s->r - 2 * rh;
   const long long entries = (long long)s->T * (rt / 2) + (long long)(s->Hg + s->W) * (rh / 2);
   return entries <= pairk::kTabCap;
@@ -786,6 +822,7 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
   prm.z_glb = z_glb;
   prm.gate = gate;
   prm.out = out;
+  prm.out_32b = rola_host::aligned(out, 32) ? 1 : 0;
   prm.dev_err = dev_err;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
   {

@@ -255,3 +255,24 @@ def test_layer_entry_points(cfg):
     assert torch.equal(out3, out)
     assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0
     assert rb.layer_launches(shape) in (5, 6)
+
+
+def test_attention_output_alignment_16_bytes():
+    """The output may be 16-byte aligned only (the epilogue then stores 16
+    bytes at a time instead of 32): same result either way."""
+    w = synth.custom_workload(synth.WORKLOADS[2], H=2)
+    inp = synth.make_inputs(w)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx = rb.select_blocks(shape, q, k)
+    states = rb.block_states(shape, k, v, P)
+    ref = rb.attention_fwd(shape, q, k, v, idx, P, states, gate)
+    n = ref.numel()
+    raw = torch.empty(n + 64, dtype=torch.bfloat16, device="cuda")
+    base = raw.data_ptr()
+    off = ((32 - base % 32) % 32 + 16) // 2  # elements to a 16-mod-32 address
+    out = raw[off:off + n].view(ref.shape)
+    assert out.data_ptr() % 32 == 16
+    rb.attention_fwd(shape, q, k, v, idx, P, states, gate, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
