@@ -115,8 +115,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint16_t* sP = reinterpret_cast<uint16_t*>(smem + Ly::pt_off);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t4 = lane & 3;
-  const int my_items =
-      p.items > (int)blockIdx.x ? (p.items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // each CTA takes a contiguous run of items (consecutive blocks of one head,
+  // so that P_h rarely changes)
+  const int per_cta = (p.items + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int first_item = (int)blockIdx.x * per_cta;
+  const int my_items = max(0, min(per_cta, p.items - first_item));
 
   if (tid == 0) {
     mbar_init(&M.full, 1);
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   volatile int* abort = &M.abort;
 
   auto decode = [&](int it, int& b, int& h, int& blk) {
-    const int id = (int)blockIdx.x + it * (int)gridDim.x;
+    const int id = first_item + it;
     blk = id % p.nb;
     h = (id / p.nb) % p.H;
     b = id / (p.nb * p.H);
