@@ -72,41 +72,69 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 
 // ---------------------------------------------------------------- scores
 // sigma[b,h,a,j] = qbar[b,h,a,:] . kbar[b,h,j,:] / sqrt(d) in float64.
-// CTA tile 64 x 64 (4 warps of 32 x 32), d staged through shared memory in
-// chunks of 32; each warp runs 4 x 4 DMMA m8n8k4 tiles per k-step of 4.
+// CTA tile 64 x 64 (4 warps of 32 x 32); d is staged through shared memory in
+// chunks of 32 by asynchronous copies (cp.async, two stages: the next chunk
+// lands while the DMMA m8n8k4 tiles run on the current one); rows past
+// n_blocks are zero-filled by the copy.
 constexpr int kScTile = 64, kScChunk = 32, kScStride = 36;  // stride keeps DMMA loads conflict-free
+constexpr int kScStageDoubles = 2 * kScTile * kScStride;     // A and B chunk of one stage
+constexpr size_t kScSmemBytes = 2 * kScStageDoubles * sizeof(double);
 
 ROLA_DEV void dmma_8x8x4(double (&c)[2], double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                : "+d"(c[0]), "+d"(c[1])
                : "d"(a), "d"(b));
 }
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+ROLA_DEV void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+ROLA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+ROLA_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar,
                                                     const double* __restrict__ kbar,
                                                     double* __restrict__ sigma, int H, int d,
                                                     int nb) {
-  __shared__ double sA[kScTile * kScStride];
-  __shared__ double sB[kScTile * kScStride];
+  extern __shared__ double sc_smem[];  // [2 stages][A | B][kScTile * kScStride]
   const int bh = blockIdx.z;
   const int row0 = blockIdx.y * kScTile, col0 = blockIdx.x * kScTile;
   const double* A = qbar + (size_t)bh * nb * d;
   const double* Bm = kbar + (size_t)bh * nb * d;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wr = (warp >> 1) * 32, wc = (warp & 1) * 32;
+  // chunk c0 of both operands into stage st: 64 rows x 16 pieces of 16 bytes each
+  auto load = [&](int st, int c0) {
+    double* sA = sc_smem + st * kScStageDoubles;
+    double* sB = sA + kScTile * kScStride;
+    for (int e = threadIdx.x; e < kScTile * (kScChunk / 2); e += blockDim.x) {
+      const int r = e / (kScChunk / 2), c = (e % (kScChunk / 2)) * 2;
+      const bool ra = row0 + r < nb, rb = col0 + r < nb;
+      cp_async16(sA + r * kScStride + c, ra ? A + (size_t)(row0 + r) * d + c0 + c : A, ra ? 16u : 0u);
+      cp_async16(sB + r * kScStride + c, rb ? Bm + (size_t)(col0 + r) * d + c0 + c : Bm, rb ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
   double acc[4][4][2];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
 
-  for (int c0 = 0; c0 < d; c0 += kScChunk) {
-    for (int e = threadIdx.x; e < kScTile * kScChunk; e += blockDim.x) {
-      const int r = e / kScChunk, c = e % kScChunk;
-      sA[r * kScStride + c] = (row0 + r < nb) ? A[(size_t)(row0 + r) * d + c0 + c] : 0.0;
-      sB[r * kScStride + c] = (col0 + r < nb) ? Bm[(size_t)(col0 + r) * d + c0 + c] : 0.0;
+  const int nchunks = d / kScChunk;
+  load(0, 0);
+  for (int ch = 0; ch < nchunks; ++ch) {
+    if (ch + 1 < nchunks) {
+      load((ch + 1) & 1, (ch + 1) * kScChunk);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const double* sA = sc_smem + (ch & 1) * kScStageDoubles;
+    const double* sB = sA + kScTile * kScStride;
 #pragma unroll
     for (int kk = 0; kk < kScChunk; kk += 4) {
       double af[4], bf[4];
@@ -120,7 +148,7 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
 #pragma unroll
         for (int j = 0; j < 4; ++j) dmma_8x8x4(acc[i][j], af[i], bf[j]);
     }
-    __syncthreads();
+    __syncthreads();  // stage (ch & 1) is refilled by the load two chunks on
   }
   const double rs = sqrt((double)d);
   double* S = sigma + (size_t)bh * nb * nb;
@@ -284,7 +312,10 @@ rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, cons
                                  double* sigma, int32_t* idx, cudaStream_t cs) {
   const int nb = rola_num_blocks(s);
   const int tiles = (nb + kScTile - 1) / kScTile;
-  score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, 0, cs>>>(qbar, kbar, sigma, s->H, s->d, nb);
+  if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScSmemBytes) !=
+      cudaSuccess)
+    return ROLA_ERR_CUDA;
+  score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, kScSmemBytes, cs>>>(qbar, kbar, sigma, s->H, s->d, nb);
   const int rows = s->B * s->H * nb;
   const int nper = (nb + 31) / 32;
   if (nper <= 4) launch_topk<4>(sigma, idx, rows, nb, s->k_b, cs);
