@@ -151,6 +151,27 @@ def cpu_baseline(w, inp) -> dict:
             "sample": text + f"; {dt:.1f} s"}
 
 
+# ---------------------------------------------------------------- replicas
+
+def max_over_ranks(x: float) -> float:
+    """Max of a per-rank scalar over the process group (the value itself when
+    there is none): multi-GPU times are the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flop_per_step: float, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job TFLOP/s of `world` replicas that each ran `steps` steps of
+    `flop_per_step`, timed by the slowest rank's `total_ms`."""
+    return world * flop_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args) -> int:
@@ -236,14 +257,10 @@ def run_gpu(args) -> int:
 
     per_stage = {nm: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)]
                  for i, nm in enumerate(stage_names)}
-    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[K - 1][2]))
     ms_step = total_ms / K
     flop = w.sparse_flops()
-    value = world * flop * K / (total_ms * 1e-3) / 1e12
+    value = job_tflops(flop, K, world, total_ms)
 
     # one FP8 W8A8 projection of the full attention block (x [N, 5120] ->
     # [N, 5120]: quantisation + tcgen05 GEMM), timed on its own after the layer
@@ -267,12 +284,8 @@ def run_gpu(args) -> int:
             hl(*host, out_h)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / K2
-        t2 = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(t2, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t2.item())
-        e2e = {"value": world * flop / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / K2)
+        e2e = {"value": job_tflops(flop, 1, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in host),
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size()}
 
