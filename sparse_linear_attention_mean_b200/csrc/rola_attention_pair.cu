@@ -147,15 +147,12 @@ ROLA_DEV void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %
 template <uint32_t N>
 ROLA_DEV void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 
-// Read-only 16-byte load that does not allocate in L1: the block states are
-// read once per unit and would only evict other lines (measured: ~4 % of the
-// kernel's time on the 14B-720P layer).
-ROLA_DEV float4 ldg_na(const float4* p) {
-  float4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+// 32-byte read-only load (two float4) that does not allocate in L1: the block
+// states are read once per unit and would only evict other lines.
+ROLA_DEV void ldg_na8(const float* p, float4& a, float4& b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(a.x), "=f"(a.y), "=f"(a.z), "=f"(a.w), "=f"(b.x), "=f"(b.y), "=f"(b.z), "=f"(b.w)
                : "l"(p));
-  return r;
 }
 
 ROLA_DEV void decode_unit(const Params& p, int id, int& b, int& h, int& pair) {
@@ -445,14 +442,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           mbar_arrive(&M.pt_full);
         }
-        // each thread owns float4 entries t + 64 i of both accumulators
+        // Thread t owns accumulator slots t + 64 i (float4, i < PER) of both
+        // slots' accumulators; slot i holds the four state elements at
+        // 8 (t + 64 (i / 2)) + 4 (i % 2), so that a state is read with 32-byte
+        // loads (two slots each) while the shared-memory slots stay
+        // contiguous across the warp.
         {
-          const float4* Sg = reinterpret_cast<const float4*>(p.S_glb + bh * R * D);
+          const float* Sg = p.S_glb + bh * R * D;
 #pragma unroll
-          for (int i = 0; i < PER; ++i) {
-            const float4 g4 = __ldg(Sg + t + 64 * i);
-            accs[t + 64 * i] = g4;
-            accs[R * D / 4 + t + 64 * i] = g4;
+          for (int i2 = 0; i2 < PER / 2; ++i2) {
+            float4 g0, g1;
+            ldg_na8(Sg + 8 * (t + 64 * i2), g0, g1);
+            accs[t + 64 * (2 * i2)] = g0;
+            accs[t + 64 * (2 * i2 + 1)] = g1;
+            accs[R * D / 4 + t + 64 * (2 * i2)] = g0;
+            accs[R * D / 4 + t + 64 * (2 * i2 + 1)] = g1;
           }
         }
         const float zg = t < R ? p.z_glb[bh * R + t] : 0.f;
@@ -463,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int mk = U.umask[j];
           float4 xv[PER];
 #pragma unroll
-          for (int i = 0; i < PER; ++i) xv[i] = ldg_na(src + t + 64 * i);
+          for (int i2 = 0; i2 < PER / 2; ++i2)
+            ldg_na8(reinterpret_cast<const float*>(src) + 8 * (t + 64 * i2), xv[2 * i2], xv[2 * i2 + 1]);
           const float zv = t < R ? __ldg(p.z_blk + st * R + t) : 0.f;
 #pragma unroll
           for (int sl = 0; sl < 2; ++sl) {
@@ -498,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t h01 = pack_bf16(v[i].x, v[i].y), h23 = pack_bf16(v[i].z, v[i].w);
             const uint32_t l01 = pack_bf16(v[i].x - bf16_lo(h01), v[i].y - bf16_hi(h01));
             const uint32_t l23 = pack_bf16(v[i].z - bf16_lo(h23), v[i].w - bf16_hi(h23));
-            const int f = (t + 64 * i) * 4;
+            const int f = 8 * (t + 64 * (i >> 1)) + 4 * (i & 1);
             const int c = f / D, e = f % D;
             const uint32_t off = (e >> 6) * (R * 128) + (c >> 3) * 1024 + (c & 7) * 128 +
                                  ((((e & 63) >> 3) ^ (c & 7)) << 4) + (e & 7) * 2;

@@ -276,3 +276,24 @@ def test_attention_output_alignment_16_bytes():
     rb.attention_fwd(shape, q, k, v, idx, P, states, gate, out=out)
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+def test_attention_states_16_byte_aligned():
+    """Block states that are 16- but not 32-byte aligned take the one-tile
+    kernel (the two-tile kernel reads them 32 bytes at a time): same result
+    within the output tolerance."""
+    w = synth.custom_workload(synth.WORKLOADS[2], H=2)
+    inp = synth.make_inputs(w)
+    shape = rb.Shape.of(w)
+    q, k, v, P, gate = dev_inputs(inp)
+    idx = rb.select_blocks(shape, q, k)
+    S_blk, z_blk, S_glb, z_glb = rb.block_states(shape, k, v, P)
+    ref = rb.attention_fwd(shape, q, k, v, idx, P, (S_blk, z_blk, S_glb, z_glb), gate)
+    raw = torch.empty(S_blk.numel() + 16, dtype=torch.float32, device="cuda")
+    off = ((32 - raw.data_ptr() % 32) % 32 + 16) // 4
+    S16 = raw[off:off + S_blk.numel()].view(S_blk.shape)
+    S16.copy_(S_blk)
+    assert S16.data_ptr() % 32 == 16
+    out = rb.attention_fwd(shape, q, k, v, idx, P, (S16, z_blk, S_glb, z_glb), gate)
+    torch.cuda.synchronize()
+    check_close(bf16_to_f64(out), bf16_to_f64(ref), atol=2e-2, rtol=2e-2, what="16-byte aligned states")
