@@ -476,12 +476,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             float4* a = accs + sl * (R * D / 4);
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
-              float4 v = a[t + 64 * i];
-              v.x -= xv[i].x;
-              v.y -= xv[i].y;
-              v.z -= xv[i].z;
-              v.w -= xv[i].w;
-              a[t + 64 * i] = v;
+              // packed f32x2 subtractions: half the instructions
+              const float4 v = a[t + 64 * i];
+              float r0, r1, r2, r3;
+              f32x2_split(fsub2(f32x2(v.x, v.y), f32x2(xv[i].x, xv[i].y)), r0, r1);
+              f32x2_split(fsub2(f32x2(v.z, v.w), f32x2(xv[i].z, xv[i].w)), r2, r3);
+              a[t + 64 * i] = make_float4(r0, r1, r2, r3);
             }
             zs[sl] -= zv;
           }
