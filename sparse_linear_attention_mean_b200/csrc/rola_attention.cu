@@ -631,8 +631,9 @@ extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_
   prm.dev_err = dev_err;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  // the two-tile kernel reads the states with 32-byte loads
-  if (pair_kernel_supports(s) && rola_host::aligned(S_blk, 32) && rola_host::aligned(S_glb, 32))
+  // the two-tile kernel reads the states with 32-byte loads and P_h with 16-byte loads
+  if (pair_kernel_supports(s) && rola_host::aligned(S_blk, 32) && rola_host::aligned(S_glb, 32) &&
+      rola_host::aligned(P, 16))
     return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, cs);
   if (s->d == 128 && s->block == 128 && s->r == 32) return launch_attn<128, 128, 32>(s, q, k, v, prm, cs);
   if (s->d == 128 && s->block == 128 && s->r == 16) return launch_attn<128, 128, 16>(s, q, k, v, prm, cs);

@@ -414,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // linear-branch MMA (N = d, K = r, 128-byte swizzle).
       const int t = tid - 320;  // 0..63
       constexpr int PER = R * D / 256;  // float4 of a block state per thread
+      int pt_head = -1;  // head whose P_h^T the shared-memory operand holds
       float4* accs = reinterpret_cast<float4*>(smem + Ly::acc_off);  // [2][R*D/4]
       uint32_t uc[2] = {0, 0};
       bool ok = true;
@@ -429,17 +430,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < 2; ++s)
           if (ok && uc[s] >= 1) ok = warp_wait(&M.l_done[s], (uc[s] - 1) & 1, abort);
         if (!ok) break;
-        // P_h^T (K-major, N = r rows, K = d, 128-byte swizzle)
+        // P_h^T (K-major, N = r rows, K = d, 128-byte swizzle), rewritten only
+        // when the head changes; P_h is read 8 values (16 bytes) at a time
         {
-          uint8_t* pt = smem + Ly::pt_off;
-          for (int e = t; e < R * D; e += 64) {
-            const int c = e / R, rr = e % R;
-            const uint16_t val = p.P[((size_t)h * D + c) * R + rr];
-            const int byte = (c & 63) * 2;
-            const int chunk = (byte >> 4) ^ (rr & 7);
-            *reinterpret_cast<uint16_t*>(pt + (c >> 6) * (32 * 128) + rr * 128 + chunk * 16 + (byte & 15)) = val;
+          if (h != pt_head) {
+            uint8_t* pt = smem + Ly::pt_off;
+            for (int e8 = t; e8 < R * D / 8; e8 += 64) {
+              const int c = e8 / (R / 8), r0 = (e8 % (R / 8)) * 8;
+              const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.P + ((size_t)h * D + c) * R + r0));
+              const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+              const int byte = (c & 63) * 2;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int rr = r0 + j;
+                const int chunk = (byte >> 4) ^ (rr & 7);
+                *reinterpret_cast<uint16_t*>(pt + (c >> 6) * (32 * 128) + rr * 128 + chunk * 16 + (byte & 15)) =
+                    (uint16_t)(wv[j >> 1] >> (16 * (j & 1)));
+              }
+            }
+            fence_proxy_async_smem();
+            pt_head = h;
           }
-          fence_proxy_async_smem();
           mbar_arrive(&M.pt_full);
         }
         // Thread t owns accumulator slots t + 64 i (float4, i < PER) of both
