@@ -424,6 +424,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const UnitList& U = M.L[buf];
         const int b = U.b, h = U.h;
         const size_t bh = (size_t)b * p.H + h;
+        // The global state, where both accumulators start, is requested
+        // before the wait below so that its latency hides behind it.  Thread t
+        // owns accumulator slots t + 64 i (float4, i < PER) of both slots'
+        // accumulators; slot i holds the four state elements at
+        // 8 (t + 64 (i / 2)) + 4 (i % 2), so that a state is read with 32-byte
+        // loads (two slots each) while the shared-memory slots stay contiguous
+        // across the warp.
+        float4 g4[PER];
+#pragma unroll
+        for (int i2 = 0; i2 < PER / 2; ++i2)
+          ldg_na8(p.S_glb + bh * R * D + 8 * (t + 64 * i2), g4[2 * i2], g4[2 * i2 + 1]);
         // the previous unit's linear-branch MMAs read these accumulators
         // (and its q P_h MMAs read P_h^T) -- wait for them
 #pragma unroll
@@ -453,22 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive(&M.pt_full);
         }
-        // Thread t owns accumulator slots t + 64 i (float4, i < PER) of both
-        // slots' accumulators; slot i holds the four state elements at
-        // 8 (t + 64 (i / 2)) + 4 (i % 2), so that a state is read with 32-byte
-        // loads (two slots each) while the shared-memory slots stay
-        // contiguous across the warp.
-        {
-          const float* Sg = p.S_glb + bh * R * D;
 #pragma unroll
-          for (int i2 = 0; i2 < PER / 2; ++i2) {
-            float4 g0, g1;
-            ldg_na8(Sg + 8 * (t + 64 * i2), g0, g1);
-            accs[t + 64 * (2 * i2)] = g0;
-            accs[t + 64 * (2 * i2 + 1)] = g1;
-            accs[R * D / 4 + t + 64 * (2 * i2)] = g0;
-            accs[R * D / 4 + t + 64 * (2 * i2 + 1)] = g1;
-          }
+        for (int i = 0; i < PER; ++i) {
+          accs[t + 64 * i] = g4[i];
+          accs[R * D / 4 + t + 64 * i] = g4[i];
         }
         const float zg = t < R ? p.z_glb[bh * R + t] : 0.f;
         float zs[2] = {zg, zg};
