@@ -232,7 +232,9 @@ def run_gpu(args) -> int:
     # the layer's own entry point; three events split it into its two stages
     layer = rb.Layer(shape)
     out = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device="cuda")
-    stage_names = ("select+states", "attention")
+    # five events: the q/k/v pass (block means + states), scores + top-k,
+    # state totals, attention
+    stage_names = ("prep", "score+topk", "state_totals", "attention")
     launches_per_step = rb.layer_launches(shape)
 
     for _ in range(args.warmup):
@@ -243,7 +245,7 @@ def run_gpu(args) -> int:
     torch.cuda.synchronize()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
     with ClockSampler(local) as clk:
         time.sleep(0.3)
         for s in range(K):
@@ -257,7 +259,7 @@ def run_gpu(args) -> int:
 
     per_stage = {nm: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(K)]
                  for i, nm in enumerate(stage_names)}
-    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[K - 1][2]))
+    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[K - 1][4]))
     ms_step = total_ms / K
     flop = w.sparse_flops()
     value = job_tflops(flop, K, world, total_ms)
@@ -306,6 +308,7 @@ def run_gpu(args) -> int:
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {**workload_config(w), "parallelism": f"replicas x{world}"},
             "kernels_ms": {nm: statistics.mean(x) for nm, x in per_stage.items()},
+            "hbm": hbm_report(w, {nm: statistics.mean(x) for nm, x in per_stage.items()}, peaks),
             "attention_tflops": achieved,
             "layer_frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
             "roofline": {"bound": "tensor", "kernel": "rola_attn_pair_kernel", "achieved": achieved,
@@ -324,6 +327,21 @@ def run_gpu(args) -> int:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def hbm_report(w, stage_ms: dict, peaks: dict) -> dict:
+    """Achieved HBM bandwidth of the HBM-bound stages from their algorithmic
+    bytes: the pass over q, k, v (reads q, k, v; writes the block states and
+    the float64 block means) and the state totals (read the block states)."""
+    act = 2.0 * w.B * w.N * w.H * w.d
+    states = 4.0 * w.B * w.H * w.n_blocks * w.r * (w.d + 1)
+    means = 2.0 * 8 * w.B * w.H * w.n_blocks * w.d
+    out = {"peak_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth"}
+    for nm, nbytes in (("prep", 3 * act + states + means), ("state_totals", states)):
+        if nm in stage_ms and stage_ms[nm] > 0:
+            gbs = nbytes / (stage_ms[nm] * 1e-3) / 1e9
+            out[nm] = {"bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+    return out
 
 
 def fp8_projection(M: int, D: int, stream, reps: int = 5) -> dict:

@@ -177,14 +177,22 @@ rola_status_t rola_layer_fwd(const rola_shape_t* shape, const uint16_t* q, const
                              void* stream);
 
 /* rola_layer_fwd with CUDA events recorded on `stream` at its stage
- * boundaries, for profiling: events[0] before the first kernel, events[1]
- * once the selection and the block states are done, events[2] after the
- * attention kernel.  `events` points to three cudaEvent_t the caller created
- * (or is NULL, which makes the call identical to rola_layer_fwd). */
+ * boundaries, for profiling.  `events` points to n_events cudaEvent_t the
+ * caller created (or is NULL, which makes the call identical to
+ * rola_layer_fwd; n_events is then ignored):
+ *   n_events = 3: before the first kernel, once the selection and the block
+ *                 states are done, after the attention kernel;
+ *   n_events = 5: before the first kernel, after the pass over q, k, v
+ *                 (block means and states), after the scores and top-k,
+ *                 after the state totals, after the attention kernel.
+ * (For shapes without the fused pass, the second event follows the
+ * selector and the fourth the block states.)  Other counts:
+ * ROLA_ERR_INVALID_ARG. */
 rola_status_t rola_layer_fwd_timed(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
                                    const uint16_t* v, const uint16_t* P, const float* gate,
                                    uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
-                                   int32_t* dev_err, void* stream, void* const* events);
+                                   int32_t* dev_err, void* stream, void* const* events,
+                                   int32_t n_events);
 
 /* Number of kernels one rola_layer_fwd call launches for `shape` (0 for an
  * invalid or unsupported shape); memory copies are not counted. */

@@ -106,7 +106,7 @@ def lib() -> ctypes.CDLL:
         L.rola_layer_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         L.rola_layer_fwd_timed.restype = ctypes.c_int
         L.rola_layer_fwd_timed.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp,
-                                           ctypes.POINTER(ctypes.c_void_p)]
+                                           ctypes.POINTER(ctypes.c_void_p), i32]
         L.rola_layer_kernel_launches.restype = ctypes.c_int
         L.rola_layer_kernel_launches.argtypes = [sp]
         L.rola_layer_fwd_host.restype = ctypes.c_int
@@ -241,8 +241,10 @@ class Layer:
         self.dev_err = torch.zeros(1, dtype=torch.int32, device=device)
 
     def __call__(self, q, k, v, P, gate, *, out=None, idx_out=None, stream=None, events=None):
-        """events: optional three torch.cuda.Event(enable_timing=True), recorded
-        before the layer, after selection + states, and after the attention."""
+        """events: optional three or five torch.cuda.Event(enable_timing=True):
+        three are recorded before the layer, after selection + states and after
+        the attention; five also split the first stage into the pass over q, k,
+        v, the scores + top-k and the state totals."""
         s = self.shape
         act = (s.B, s.N, s.H, s.d)
         for t, nm in ((q, "q"), (k, "k"), (v, "v")):
@@ -259,15 +261,16 @@ class Layer:
                                         self.ws_bytes, _ptr(self.dev_err), _stream(stream)),
                    "rola_layer_fwd")
         else:
-            if len(events) != 3:
-                raise ValueError("events: three torch.cuda.Event")
+            if len(events) not in (3, 5):
+                raise ValueError("events: three or five torch.cuda.Event")
             for e in events:
                 if not e.cuda_event:  # torch creates the handle on first record
                     e.record(stream if stream is not None else torch.cuda.current_stream())
-            ev = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
+            ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
             _check(lib().rola_layer_fwd_timed(ctypes.byref(self.c), _ptr(q), _ptr(k), _ptr(v), _ptr(P),
                                               _ptr(gate), _ptr(out), _ptr(idx_out), _ptr(self.ws),
-                                              self.ws_bytes, _ptr(self.dev_err), _stream(stream), ev),
+                                              self.ws_bytes, _ptr(self.dev_err), _stream(stream), ev,
+                                              len(events)),
                    "rola_layer_fwd_timed")
         return out
 

@@ -164,17 +164,22 @@ extern "C" rola_status_t rola_layer_fwd(const rola_shape_t* s, const uint16_t* q
                                         const uint16_t* v, const uint16_t* P, const float* gate,
                                         uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
                                         int32_t* dev_err, void* stream) {
-  return rola_layer_fwd_timed(s, q, k, v, P, gate, out, idx_out, ws, ws_bytes, dev_err, stream, nullptr);
+  return rola_layer_fwd_timed(s, q, k, v, P, gate, out, idx_out, ws, ws_bytes, dev_err, stream, nullptr, 0);
 }
 
 extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint16_t* q,
                                               const uint16_t* k, const uint16_t* v, const uint16_t* P,
                                               const float* gate, uint16_t* out, int32_t* idx_out,
                                               void* ws, size_t ws_bytes, int32_t* dev_err, void* stream,
-                                              void* const* events) {
-  auto mark = [&](int i) -> bool {
-    return !events || cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]),
-                                      reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess;
+                                              void* const* events, int32_t n_events) {
+  if (events && n_events != 3 && n_events != 5) return ROLA_ERR_INVALID_ARG;
+  // stage boundaries 0..4 (start, after the q/k/v pass, after scores and
+  // top-k, after the totals, end); three events keep stages 0, 3 and 4
+  auto mark = [&](int stage) -> bool {
+    if (!events) return true;
+    const int i = n_events == 5 ? stage : (stage == 0 ? 0 : stage == 3 ? 1 : stage == 4 ? 2 : -1);
+    return i < 0 || cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]),
+                                    reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess;
   };
   rola_status_t st = check_shape(s);
   if (st != ROLA_OK) return st;
@@ -201,21 +206,24 @@ extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint1
     double* sigma = reinterpret_cast<double*>(base + L.select + round_up(2 * pooled * sizeof(double), 256));
     st = rola::launch_prep_kernel(s, q, k, v, P, qbar, kbar, S_blk, z_blk, dev_err, cs);
     if (st != ROLA_OK) return st;
+    if (!mark(1)) return ROLA_ERR_CUDA;
     st = rola::select_from_pooled(s, qbar, kbar, sigma, idx, cs);
     if (st != ROLA_OK) return st;
+    if (!mark(2)) return ROLA_ERR_CUDA;
     st = rola::launch_states_total(s, S_blk, z_blk, S_glb, z_glb, cs);
     if (st != ROLA_OK) return st;
   } else {
     st = rola_select_blocks(s, q, k, idx, nullptr, base + L.select, L.idx - L.select, stream);
     if (st != ROLA_OK) return st;
+    if (!mark(1) || !mark(2)) return ROLA_ERR_CUDA;
     st = rola_block_states(s, k, v, P, S_blk, z_blk, S_glb, z_glb, stream);
     if (st != ROLA_OK) return st;
   }
-  if (!mark(1)) return ROLA_ERR_CUDA;
+  if (!mark(3)) return ROLA_ERR_CUDA;
   st = rola_attention_fwd(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
                           stream);
   if (st != ROLA_OK) return st;
-  if (!mark(2)) return ROLA_ERR_CUDA;
+  if (!mark(4)) return ROLA_ERR_CUDA;
   if (idx_out) {
     const size_t bytes = (size_t)s->B * s->H * rola_num_blocks(s) * s->k_b * sizeof(int32_t);
     if (cudaMemcpyAsync(idx_out, idx, bytes, cudaMemcpyDeviceToDevice,

@@ -91,3 +91,11 @@ def test_fp8_gemm_arguments_rejected_on_host(lib):
     assert gemm(64, 64, 64, odd, ok, ok, ok, ok, None, None) == 5   # misaligned codes
     assert gemm(64, 64, 64, ok, ok, ok, odd, ok, None, None) == 5   # misaligned w_scale
     assert lib.fp8_linear_w8a8(64, 64, 64, ok, ok, ok, ok, None, 0, None, None) == 3  # no workspace
+
+
+def test_timed_layer_event_count_checked_on_host(lib):
+    cs = rb.Shape(1, 2, 64, 4, 16, 16, 64, 4, 16).c()
+    ok = ctypes.c_void_p(4096)
+    ev = (ctypes.c_void_p * 4)(4096, 4096, 4096, 4096)
+    st = lib.rola_layer_fwd_timed(ctypes.byref(cs), ok, ok, ok, ok, ok, ok, None, ok, 1 << 30, None, None, ev, 4)
+    assert st == 1  # ROLA_ERR_INVALID_ARG: three or five events
