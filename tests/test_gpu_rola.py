@@ -190,8 +190,15 @@ def test_dense_limit_s0(block, d, r):
     check_close(bf16_to_f64(out), ref, what="dense limit vs SDPA")
 
 
-def test_batch_two_matches_single():
-    w = synth.custom_workload(synth.WORKLOADS[0], B=2)
+@pytest.mark.parametrize("base", ["tiny", "128"])
+def test_batch_two_matches_single(base):
+    """B = 2 through the selector, the states and the attention: the 64-token
+    workload (one-tile kernel) and a 128-token-block one (two-tile kernel,
+    fused prep pass on the layer path)."""
+    if base == "tiny":
+        w = synth.custom_workload(synth.WORKLOADS[0], B=2)
+    else:
+        w = synth.Workload("batch2-128", 2, 3, 128, 2, 16, 20, 128, 0, 2, 32, seed=9)
     inp = synth.make_inputs(w)
     idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
     shape = rb.Shape.of(w)
@@ -199,6 +206,15 @@ def test_batch_two_matches_single():
     idx_gpu = rb.select_blocks(shape, q, k).cpu().numpy()
     assert np.array_equal(idx_gpu, idx_ref)
     _attention_case(w, inp, heads=None, qblocks=None)
+    # the whole layer: the same mask, and the output matches the oracle
+    layer = rb.Layer(shape)
+    idx_l = torch.empty_like(torch.from_numpy(idx_ref)).cuda()
+    out = layer(q, k, v, P, gate, idx_out=idx_l)
+    torch.cuda.synchronize()
+    assert int(layer.dev_err.item()) == 0
+    assert np.array_equal(idx_l.cpu().numpy(), idx_ref)
+    res = ro.rola_forward(inp, bs=w.block, k_b=w.k_b, grid=_grid(w), rope_base=w.rope_base, idx=idx_ref)
+    check_close(bf16_to_f64(out), ro.assemble_output(res, w.B, w.N, w.H, w.d, w.block), what="layer, B = 2")
 
 
 def test_bad_index_reported_not_trapped():
