@@ -144,7 +144,7 @@ def blas_threads() -> int:
 
 
 def cpu_baseline(w, inp) -> dict:
-    # about 10 s of host work: every query block of four heads
+    # several seconds of host work: every query block of four heads
     heads = tuple(sorted({0, w.H // 3, (2 * w.H) // 3, w.H - 1}))
     dt, flop, text = oracle_sample(w, inp, heads=heads, qblocks=range(w.n_blocks))
     return {"value": flop / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -385,11 +385,18 @@ def fp8_projection(M: int, D: int, stream, reps: int = 5) -> dict:
 
 
 def kernel_hash() -> str:
+    """Hash of the attention kernel's source code with comments and blank
+    lines removed: it changes when the code does, not when a comment does."""
     import hashlib
+    import re
     h = hashlib.sha1()
     for nm in ("rola_attention.cu", "rola_attention_pair.cu", "rola_common.cuh"):
-        with open(os.path.join(ROOT, "sparse_linear_attention_mean_b200", "csrc", nm), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sparse_linear_attention_mean_b200", "csrc", nm)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:12]
 
 

@@ -21,13 +21,17 @@
 //                   read, and rescales O lazily (only when the row max grows
 //                   by more than 2^8, which keeps P <= 256); at the tile end
 //                   rho_q = R(t, y, x) phi(q P_h) (rotary angles from a per-CTA
-//                   cos/sin table), psi_q . z_U, and the epilogue
-//                   o = O / l + g_h * L / (psi_q . z_U)
-//   warp 8          producer: unit lists, Q tiles, K/V ring (TMA)
-//   warp 9          MMA issuer: S = Q K^T, O += P V, q P_h, L = rho_q S_U
-//   warps 10-11     head projection P_h^T to shared memory; gather of the
-//                   linear-branch states of every union block into fp32
-//                   shared-memory accumulators; S_U = S - sum_kept S_j, z_U
+//                   cos/sin table), psi_q . z_U and rho'_q (below), and the
+//                   epilogue out = O / l (tile-end code as rolled loops: it
+//                   runs once per unit, cold in the instruction cache)
+//   warp 8          producer: the unit lists, built one unit ahead by a
+//                   bitmap merge of both kept lists (three list buffers),
+//                   Q tiles and the K/V ring (TMA)
+//   warp 9          MMA issuer: S = Q K^T, O += P V, q P_h, O += rho'_q S_U
+//   warps 10-11     P_h^T in shared memory (rewritten when the head
+//                   changes); gather of the linear-branch states of every
+//                   union block (32-byte loads that skip L1) into fp32
+//                   shared-memory accumulators: S_U = S - sum_kept S_j, z_U
 // The linear branch is folded into O: at a tile end the softmax warps write
 // rho'_q = rho_q g_h l / (psi_q . z_U) (bf16 hi + lo) into tensor memory and
 // one more MMA adds rho'_q S_U to O, S_U coming from the gather warps'
