@@ -153,10 +153,15 @@ rola_status_t rola_block_states(const rola_shape_t* shape, const uint16_t* k, co
  *   idx      int32 [B, H, n_blocks, k_b], rows strictly ascending; a bad entry
  *            is skipped and sets ROLA_DEVERR_BAD_INDEX
  *   P        bf16 [H, d, r];  S_blk, z_blk, S_glb, z_glb as produced by
- *            rola_block_states;  gate  fp32 [H]
- *   out      out, bf16 [B, N, H, d]
+ *            rola_block_states (S_blk, S_glb 16-byte aligned);  gate  fp32 [H]
+ *   out      out, bf16 [B, N, H, d], 16-byte aligned
  *   dev_err  one int32 the caller zeroed; may be NULL (then device-side
- *            problems are still skipped but not reported) */
+ *            problems are still skipped but not reported)
+ * For d = 128, 128-token blocks and k_b <= 256 a persistent kernel walks pairs
+ * of adjacent query blocks over the union of their kept lists; it reads the
+ * states 32 bytes and P 16 bytes at a time, so it is chosen when S_blk and
+ * S_glb are 32-byte and P 16-byte aligned (otherwise, and for the other
+ * shapes, a one-tile kernel runs; both give the results stated above). */
 rola_status_t rola_attention_fwd(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
                                  const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                  const float* S_blk, const float* z_blk, const float* S_glb,
@@ -168,9 +173,13 @@ rola_status_t rola_attention_fwd(const rola_shape_t* shape, const uint16_t* q, c
 /* Workspace of rola_layer_fwd: selector scratch, idx and the states. */
 size_t rola_layer_workspace_bytes(const rola_shape_t* shape);
 
-/* One RoLA attention layer: rola_select_blocks, rola_block_states and
- * rola_attention_fwd back to back on `stream`, intermediates in `ws`.
- * idx_out (optional, NULL to skip) receives a copy of the kept-block index. */
+/* One RoLA attention layer: the selection, block states and attention of
+ * rola_select_blocks, rola_block_states and rola_attention_fwd back to back on
+ * `stream`, intermediates in `ws` (256-byte aligned, rola_layer_workspace_bytes
+ * bytes).  For d = 128 and 128-token blocks one pass over q, k and v computes
+ * both the block means and the block states (same results as the separate
+ * calls; q, k, v and P 16-byte aligned).  idx_out (optional, NULL to skip)
+ * receives a copy of the kept-block index. */
 rola_status_t rola_layer_fwd(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
                              const uint16_t* v, const uint16_t* P, const float* gate, uint16_t* out,
                              int32_t* idx_out, void* ws, size_t ws_bytes, int32_t* dev_err,
