@@ -1,6 +1,6 @@
-"""The FMA-pipe 2^y used for part of the softmax exponentials: replay the
-device's float32 operation sequence (constants read from the CUDA header) and
-check it against 2^y in float64.  P is rounded to bf16 (relative 2^-9)
+"""The FMA-pipe 2^y kept beside the softmax (off by default: measured slower):
+replay its float32 operation sequence, with the coefficients of our own fit
+read from rola_common.cuh, and check it against 2^y in float64.  P is rounded to bf16 (relative 2^-9)
 afterwards, so a relative error below 1e-4 is invisible in the output."""
 import os
 import re
