@@ -11,10 +11,12 @@
 // Thread 0 TMA-loads the item's k and v tiles (128-byte swizzle) while every
 // thread loads its share of the q tile straight into registers; the other
 // CTA on the SM computes meanwhile.  Per item:
+//   * K P_h with mma.sync (first: it needs only the k tile, so the q loads
+//     have this long to land);
 //   * block sums of q and k over the valid tokens in float64 (exact for bf16;
 //     rows past N are zero), divided by the count;
-//   * K P_h with mma.sync, psi = phi(.), rho = rotation by a per-CTA cos/sin
-//     table of the 3-D rotary angles, written as bf16 hi + lo;
+//   * psi = phi(K P_h), rho = rotation by a per-CTA cos/sin table of the 3-D
+//     rotary angles, written as bf16 hi + lo;
 //   * S_j^T = V^T rho with mma.sync (hi and lo parts), z_j = sum of psi.
 // The kernel is bound by HBM: 96 KB read and ~16.5 KB written per item.
 #include <math.h>
@@ -195,6 +197,29 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (!(ok = mbar_wait(&M.full, it & 1, abort))) break;
 
+    // ---- kt = K P_h : warp w owns token rows [16w, 16w + 16)
+    constexpr int NT = R / 8;
+    float acc[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+    {
+      const uint32_t kbase = smem_u32(sk), pbase = smem_u32(sP);
+      const int arow = warp * 16 + (lane & 15);
+#pragma unroll
+      for (int kk = 0; kk < D; kk += 16) {
+        uint32_t a[4];
+        ldsm_x4(a, kbase + sw_off(arow, kk + (lane >> 4) * 8));
+#pragma unroll
+        for (int nj = 0; nj < NT; nj += 2) {
+          uint32_t bb[4];
+          ldsm_x4_t(bb, pbase + ((kk + (lane & 15)) * Ly::PS + nj * 8 + (lane >> 4) * 8) * 2);
+          mma16816(acc[nj], a, bb[0], bb[1]);
+          mma16816(acc[nj + 1], a, bb[2], bb[3]);
+        }
+      }
+    }
     // ---- block sums of q and k (float64, scaled by 2^-896: the bf16 sums are
     // exact); rows past N are zero in both (q not loaded, k zero-filled by
     // the copy)
@@ -230,29 +255,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
-    // ---- kt = K P_h : warp w owns token rows [16w, 16w + 16)
-    constexpr int NT = R / 8;
-    float acc[NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-    {
-      const uint32_t kbase = smem_u32(sk), pbase = smem_u32(sP);
-      const int arow = warp * 16 + (lane & 15);
-#pragma unroll
-      for (int kk = 0; kk < D; kk += 16) {
-        uint32_t a[4];
-        ldsm_x4(a, kbase + sw_off(arow, kk + (lane >> 4) * 8));
-#pragma unroll
-        for (int nj = 0; nj < NT; nj += 2) {
-          uint32_t bb[4];
-          ldsm_x4_t(bb, pbase + ((kk + (lane & 15)) * Ly::PS + nj * 8 + (lane >> 4) * 8) * 2);
-          mma16816(acc[nj], a, bb[0], bb[1]);
-          mma16816(acc[nj + 1], a, bb[2], bb[3]);
-        }
-      }
-    }
     __syncthreads();  // pooling partials complete
     if (p.do_pool) {
       const int tile = tid >> 7, c = tid & 127;
