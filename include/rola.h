@@ -60,6 +60,8 @@ typedef enum {
 #define ROLA_DEVERR_BAD_INDEX 0x1   /* idx entry out of [0, n_blocks) or not ascending */
 #define ROLA_DEVERR_TIMEOUT 0x2     /* a bounded pipeline wait ran out                  */
 
+/* Every size is at least 1: an empty batch, head set or grid is rejected with
+ * ROLA_ERR_INVALID_ARG (there is nothing to launch). */
 typedef struct {
   int32_t B, H, d;       /* batch, heads, head dim (64 or 128)                    */
   int32_t N;             /* valid tokens; must equal T * Hg * W                   */

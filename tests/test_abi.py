@@ -55,6 +55,10 @@ def test_num_blocks_and_workspace_sizes(lib):
 
 @pytest.mark.parametrize("field,value,status", [
     ("N", 123, 1),          # N != T*Hg*W
+    ("B", 0, 1),            # empty batch
+    ("H", 0, 1),            # no heads
+    ("T", 0, 1),            # empty grid
+    ("W", -4, 1),
     ("k_b", 0, 1),
     ("k_b", 10_000, 1),
     ("r", 3, 1),            # odd rank
