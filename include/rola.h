@@ -15,13 +15,16 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - Every tensor pointer is a DEVICE pointer owned by the caller; the library
- *    never allocates device memory.  Scratch space, where needed, is a
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller (except in
+ *    rola_layer_fwd_host, which takes host buffers); the library never
+ *    allocates device memory.  Scratch space, where needed, is a
  *    caller-provided workspace whose size a *_workspace_bytes() call reports.
  *  - "bf16" buffers hold bfloat16 bit patterns (uint16_t).
  *  - Calls are asynchronous on the given stream (a cudaStream_t; NULL is the
- *    legacy default stream) and stateless; concurrent calls on different
- *    streams are safe as long as their buffers do not overlap.
+ *    legacy default stream) and stateless, apart from the two copy streams and
+ *    seven events rola_layer_fwd_host creates once per device; concurrent
+ *    calls on different streams are safe as long as their buffers do not
+ *    overlap.
  *  - Shape, pointer and alignment problems are reported synchronously as a
  *    status code and nothing is launched.  A failed launch returns
  *    ROLA_ERR_CUDA.  No C++ exception crosses this boundary.
@@ -209,16 +212,25 @@ rola_status_t rola_layer_fwd_timed(const rola_shape_t* shape, const uint16_t* q,
  * invalid or unsupported shape); memory copies are not counted. */
 int rola_layer_kernel_launches(const rola_shape_t* shape);
 
-/* Device staging the host-buffer variant needs on top of the layer
- * workspace: q, k, v, P, gate and out. */
+/* Device staging the host-buffer variant needs: P and gate of all heads, two
+ * slots of q, k, v and out for one head group, and the layer workspace of one
+ * head group. */
 size_t rola_layer_host_workspace_bytes(const rola_shape_t* shape);
 
 /* The same layer with q, k, v, P, gate and out in HOST memory (pinned for
- * asynchronous copies): copies in, runs the layer, copies the output back,
- * all on `stream`.  The call returns once the work is enqueued; the caller
- * synchronises the stream before reading `out`.  ws: device workspace of
- * rola_layer_host_workspace_bytes(shape) bytes; dev_err: device pointer or
- * NULL. */
+ * asynchronous copies).  Every (b, h) is independent, so the heads are taken
+ * in groups whose slice of a token row is at least 2 KB (8 heads of d = 128):
+ * a group's q, k, v are copied (strided rows) into one of two device slots
+ * while the previous group computes, and each group's output is copied back
+ * into its columns of out while the next one computes.  The copies run on two
+ * streams the library creates once per device; events order them after the
+ * work already on `stream`, the compute runs on `stream`, and `stream` waits
+ * for the last copy back before anything enqueued after this call.  The call
+ * returns once the work is enqueued; the caller synchronises `stream` before
+ * reading `out`.  Calls on one device are enqueued under a lock.  The result
+ * is bit-identical to rola_layer_fwd.  ws: device workspace of
+ * rola_layer_host_workspace_bytes(shape) bytes, 256-byte aligned; dev_err:
+ * device pointer or NULL. */
 rola_status_t rola_layer_fwd_host(const rola_shape_t* shape, const uint16_t* q_host,
                                   const uint16_t* k_host, const uint16_t* v_host,
                                   const uint16_t* P_host, const float* gate_host,

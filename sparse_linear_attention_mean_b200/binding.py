@@ -286,7 +286,9 @@ def layer_launches(shape: Shape) -> int:
 
 class HostLayer:
     """The layer on HOST tensors (pinned for asynchronous copies): the library
-    copies inputs in, runs the layer and copies the output back on one stream."""
+    copies the inputs in by head groups, runs the layer on each group while the
+    next one is copied in, and copies each group's output back meanwhile; the
+    given (or current) stream waits for the last copy."""
 
     def __init__(self, shape: Shape, device="cuda"):
         self.shape = shape

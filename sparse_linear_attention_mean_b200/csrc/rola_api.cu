@@ -234,23 +234,78 @@ extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint1
 }
 
 namespace {
+// The host-buffer layer runs in head groups: (batch, head) pairs are
+// independent, so while one group computes, the next group's q, k, v cross
+// PCIe and the previous group's output goes back.  A group holds heads whose
+// slice of a token row is at least 2 KB (8 heads of d = 128), so that the
+// strided copies move long rows.
+constexpr int kHostGroupRowBytes = 2048;
+
+int host_group_heads(const rola_shape_t* s) {
+  const int row = s->d * (int)sizeof(uint16_t);
+  const int hc = (kHostGroupRowBytes + row - 1) / row;
+  return hc < s->H ? hc : s->H;
+}
+
+rola_shape_t group_shape(const rola_shape_t* s, int heads) {
+  rola_shape_t g = *s;
+  g.H = heads;
+  return g;
+}
+
+// Device staging: P and gate of all heads, two slots of (q, k, v, out) of
+// one group, compact [B, N, hc, d], and the layer workspace of one group.
 struct HostWs {
-  size_t q, k, v, P, gate, out, layer, total;
+  size_t P, gate, slot[2], q, k, v, out, slot_bytes, layer, total;
 };
 HostWs host_ws(const rola_shape_t* s) {
   using rola_internal::round_up;
   HostWs w{};
-  const size_t act = (size_t)s->B * s->N * s->H * s->d * sizeof(uint16_t);
+  const rola_shape_t g = group_shape(s, host_group_heads(s));
+  const size_t act = round_up((size_t)g.B * g.N * g.H * g.d * sizeof(uint16_t), 256);
   size_t off = 0;
-  w.q = off; off += round_up(act, 256);
-  w.k = off; off += round_up(act, 256);
-  w.v = off; off += round_up(act, 256);
-  w.out = off; off += round_up(act, 256);
   w.P = off; off += round_up((size_t)s->H * s->d * s->r * sizeof(uint16_t), 256);
   w.gate = off; off += round_up((size_t)s->H * sizeof(float), 256);
-  w.layer = off; off += rola_internal::layer_ws(s).total;
+  w.q = 0; w.k = act; w.v = 2 * act; w.out = 3 * act;
+  w.slot_bytes = 4 * act;
+  w.slot[0] = off; off += w.slot_bytes;
+  w.slot[1] = off; off += w.slot_bytes;
+  w.layer = off; off += rola_internal::layer_ws(&g).total;
   w.total = off;
   return w;
+}
+
+// Copy streams and the events that order them against the caller's stream,
+// created once per device and kept for the life of the process.  Enqueueing
+// a call holds the device's lock, so concurrent calls cannot interleave their
+// event records.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in[2] = {}, done[2] = {}, out[2] = {};
+  std::mutex lock;
+};
+constexpr int kMaxDevices = 64;
+HostPipe g_pipes[kMaxDevices];
+std::mutex g_pipes_lock;
+
+HostPipe* host_pipe() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> guard(g_pipes_lock);
+  HostPipe& hp = g_pipes[dev];
+  if (!hp.ready) {
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+      ok = cudaEventCreateWithFlags(&hp.in[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.out[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return nullptr;
+    hp.ready = true;
+  }
+  return &hp;
 }
 }  // namespace
 
@@ -270,25 +325,66 @@ extern "C" rola_status_t rola_layer_fwd_host(const rola_shape_t* s, const uint16
     return ROLA_ERR_INVALID_ARG;
   const HostWs w = host_ws(s);
   if (!ws || ws_bytes < w.total || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
+  HostPipe* hp = host_pipe();
+  if (!hp) return ROLA_ERR_CUDA;
+  std::lock_guard<std::mutex> guard(hp->lock);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   char* base = reinterpret_cast<char*>(ws);
-  const size_t act = (size_t)s->B * s->N * s->H * s->d * sizeof(uint16_t);
+  const int hc = host_group_heads(s);
+  const int groups = (s->H + hc - 1) / hc;
+  const size_t rows = (size_t)s->B * s->N;
+  const size_t row_bytes = (size_t)s->H * s->d * sizeof(uint16_t);  // one token of all heads
+  const size_t head_bytes = (size_t)s->d * sizeof(uint16_t);
   const size_t pbytes = (size_t)s->H * s->d * s->r * sizeof(uint16_t);
-  if (cudaMemcpyAsync(base + w.q, q_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(base + w.k, k_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(base + w.v, v_host, act, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(base + w.P, P_host, pbytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(base + w.gate, gate_host, (size_t)s->H * sizeof(float),
-                      cudaMemcpyHostToDevice, cs) != cudaSuccess)
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // everything before this call on `stream` (e.g. the last use of ws) first
+  if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->h2d, hp->start, 0)) ||
+      !ok(cudaStreamWaitEvent(hp->d2h, hp->start, 0)))
     return ROLA_ERR_CUDA;
-  st = rola_layer_fwd(s, reinterpret_cast<uint16_t*>(base + w.q),
-                      reinterpret_cast<uint16_t*>(base + w.k),
-                      reinterpret_cast<uint16_t*>(base + w.v),
-                      reinterpret_cast<uint16_t*>(base + w.P), reinterpret_cast<float*>(base + w.gate),
-                      reinterpret_cast<uint16_t*>(base + w.out), nullptr, base + w.layer,
-                      w.total - w.layer, dev_err, stream);
-  if (st != ROLA_OK) return st;
-  if (cudaMemcpyAsync(out_host, base + w.out, act, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+  if (!ok(cudaMemcpyAsync(base + w.P, P_host, pbytes, cudaMemcpyHostToDevice, hp->h2d)) ||
+      !ok(cudaMemcpyAsync(base + w.gate, gate_host, (size_t)s->H * sizeof(float),
+                          cudaMemcpyHostToDevice, hp->h2d)))
     return ROLA_ERR_CUDA;
+  for (int gi = 0; gi < groups; ++gi) {
+    const int sl = gi & 1;
+    const int h0 = gi * hc;
+    const int heads = s->H - h0 < hc ? s->H - h0 : hc;
+    const size_t width = (size_t)heads * head_bytes;  // this group's slice of a token row
+    char* slot = base + w.slot[sl];
+    // inputs: the slot's previous group must have finished computing
+    if (gi >= 2 && !ok(cudaStreamWaitEvent(hp->h2d, hp->done[sl], 0))) return ROLA_ERR_CUDA;
+    const uint16_t* src[3] = {q_host, k_host, v_host};
+    const size_t dst_off[3] = {w.q, w.k, w.v};
+    for (int t = 0; t < 3; ++t)
+      if (!ok(cudaMemcpy2DAsync(slot + dst_off[t], width,
+                                reinterpret_cast<const char*>(src[t]) + (size_t)h0 * head_bytes,
+                                row_bytes, width, rows, cudaMemcpyHostToDevice, hp->h2d)))
+        return ROLA_ERR_CUDA;
+    if (!ok(cudaEventRecord(hp->in[sl], hp->h2d))) return ROLA_ERR_CUDA;
+    // compute on the caller's stream once the inputs are in and the slot's
+    // previous output has gone back
+    if (!ok(cudaStreamWaitEvent(cs, hp->in[sl], 0))) return ROLA_ERR_CUDA;
+    if (gi >= 2 && !ok(cudaStreamWaitEvent(cs, hp->out[sl], 0))) return ROLA_ERR_CUDA;
+    const rola_shape_t g = group_shape(s, heads);
+    st = rola_layer_fwd(&g, reinterpret_cast<uint16_t*>(slot + w.q),
+                        reinterpret_cast<uint16_t*>(slot + w.k),
+                        reinterpret_cast<uint16_t*>(slot + w.v),
+                        reinterpret_cast<uint16_t*>(base + w.P) + (size_t)h0 * s->d * s->r,
+                        reinterpret_cast<float*>(base + w.gate) + h0,
+                        reinterpret_cast<uint16_t*>(slot + w.out), nullptr, base + w.layer,
+                        w.total - w.layer, dev_err, stream);
+    if (st != ROLA_OK) return st;
+    if (!ok(cudaEventRecord(hp->done[sl], cs))) return ROLA_ERR_CUDA;
+    // output of this group back into its columns of the host rows
+    if (!ok(cudaStreamWaitEvent(hp->d2h, hp->done[sl], 0)) ||
+        !ok(cudaMemcpy2DAsync(reinterpret_cast<char*>(out_host) + (size_t)h0 * head_bytes,
+                              row_bytes, slot + w.out, width, width, rows, cudaMemcpyDeviceToHost,
+                              hp->d2h)) ||
+        !ok(cudaEventRecord(hp->out[sl], hp->d2h)))
+      return ROLA_ERR_CUDA;
+  }
+  // the caller's stream continues after the last copies back
+  for (int sl = 0; sl < 2 && sl < groups; ++sl)
+    if (!ok(cudaStreamWaitEvent(cs, hp->out[sl], 0))) return ROLA_ERR_CUDA;
   return ROLA_OK;
 }
