@@ -319,7 +319,7 @@ extern "C" rola_status_t rola_layer_fwd_host(const rola_shape_t* s, const uint16
                                              const uint16_t* P_host, const float* gate_host,
                                              uint16_t* out_host, void* ws, size_t ws_bytes,
                                              int32_t* dev_err, void* stream) {
-  rola_status_t st = check_shape(s);
+  const rola_status_t st = check_shape(s);
   if (st != ROLA_OK) return st;
   if (!q_host || !k_host || !v_host || !P_host || !gate_host || !out_host)
     return ROLA_ERR_INVALID_ARG;
@@ -341,50 +341,68 @@ extern "C" rola_status_t rola_layer_fwd_host(const rola_shape_t* s, const uint16
   if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->h2d, hp->start, 0)) ||
       !ok(cudaStreamWaitEvent(hp->d2h, hp->start, 0)))
     return ROLA_ERR_CUDA;
+  rola_status_t result = ROLA_OK;
   if (!ok(cudaMemcpyAsync(base + w.P, P_host, pbytes, cudaMemcpyHostToDevice, hp->h2d)) ||
       !ok(cudaMemcpyAsync(base + w.gate, gate_host, (size_t)s->H * sizeof(float),
                           cudaMemcpyHostToDevice, hp->h2d)))
-    return ROLA_ERR_CUDA;
-  for (int gi = 0; gi < groups; ++gi) {
+    result = ROLA_ERR_CUDA;
+  for (int gi = 0; result == ROLA_OK && gi < groups; ++gi) {
     const int sl = gi & 1;
     const int h0 = gi * hc;
     const int heads = s->H - h0 < hc ? s->H - h0 : hc;
     const size_t width = (size_t)heads * head_bytes;  // this group's slice of a token row
     char* slot = base + w.slot[sl];
     // inputs: the slot's previous group must have finished computing
-    if (gi >= 2 && !ok(cudaStreamWaitEvent(hp->h2d, hp->done[sl], 0))) return ROLA_ERR_CUDA;
+    if (gi >= 2 && !ok(cudaStreamWaitEvent(hp->h2d, hp->done[sl], 0))) {
+      result = ROLA_ERR_CUDA;
+      break;
+    }
     const uint16_t* src[3] = {q_host, k_host, v_host};
     const size_t dst_off[3] = {w.q, w.k, w.v};
-    for (int t = 0; t < 3; ++t)
-      if (!ok(cudaMemcpy2DAsync(slot + dst_off[t], width,
-                                reinterpret_cast<const char*>(src[t]) + (size_t)h0 * head_bytes,
-                                row_bytes, width, rows, cudaMemcpyHostToDevice, hp->h2d)))
-        return ROLA_ERR_CUDA;
-    if (!ok(cudaEventRecord(hp->in[sl], hp->h2d))) return ROLA_ERR_CUDA;
+    bool copied = true;
+    for (int t = 0; copied && t < 3; ++t)
+      copied = ok(cudaMemcpy2DAsync(slot + dst_off[t], width,
+                                    reinterpret_cast<const char*>(src[t]) + (size_t)h0 * head_bytes,
+                                    row_bytes, width, rows, cudaMemcpyHostToDevice, hp->h2d));
+    if (!copied || !ok(cudaEventRecord(hp->in[sl], hp->h2d))) {
+      result = ROLA_ERR_CUDA;
+      break;
+    }
     // compute on the caller's stream once the inputs are in and the slot's
     // previous output has gone back
-    if (!ok(cudaStreamWaitEvent(cs, hp->in[sl], 0))) return ROLA_ERR_CUDA;
-    if (gi >= 2 && !ok(cudaStreamWaitEvent(cs, hp->out[sl], 0))) return ROLA_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(cs, hp->in[sl], 0)) ||
+        (gi >= 2 && !ok(cudaStreamWaitEvent(cs, hp->out[sl], 0)))) {
+      result = ROLA_ERR_CUDA;
+      break;
+    }
     const rola_shape_t g = group_shape(s, heads);
-    st = rola_layer_fwd(&g, reinterpret_cast<uint16_t*>(slot + w.q),
-                        reinterpret_cast<uint16_t*>(slot + w.k),
-                        reinterpret_cast<uint16_t*>(slot + w.v),
-                        reinterpret_cast<uint16_t*>(base + w.P) + (size_t)h0 * s->d * s->r,
-                        reinterpret_cast<float*>(base + w.gate) + h0,
-                        reinterpret_cast<uint16_t*>(slot + w.out), nullptr, base + w.layer,
-                        w.total - w.layer, dev_err, stream);
-    if (st != ROLA_OK) return st;
-    if (!ok(cudaEventRecord(hp->done[sl], cs))) return ROLA_ERR_CUDA;
+    result = rola_layer_fwd(&g, reinterpret_cast<uint16_t*>(slot + w.q),
+                            reinterpret_cast<uint16_t*>(slot + w.k),
+                            reinterpret_cast<uint16_t*>(slot + w.v),
+                            reinterpret_cast<uint16_t*>(base + w.P) + (size_t)h0 * s->d * s->r,
+                            reinterpret_cast<float*>(base + w.gate) + h0,
+                            reinterpret_cast<uint16_t*>(slot + w.out), nullptr, base + w.layer,
+                            w.total - w.layer, dev_err, stream);
+    if (result != ROLA_OK) break;
+    if (!ok(cudaEventRecord(hp->done[sl], cs))) {
+      result = ROLA_ERR_CUDA;
+      break;
+    }
     // output of this group back into its columns of the host rows
     if (!ok(cudaStreamWaitEvent(hp->d2h, hp->done[sl], 0)) ||
         !ok(cudaMemcpy2DAsync(reinterpret_cast<char*>(out_host) + (size_t)h0 * head_bytes,
                               row_bytes, slot + w.out, width, width, rows, cudaMemcpyDeviceToHost,
                               hp->d2h)) ||
-        !ok(cudaEventRecord(hp->out[sl], hp->d2h)))
-      return ROLA_ERR_CUDA;
+        !ok(cudaEventRecord(hp->out[sl], hp->d2h))) {
+      result = ROLA_ERR_CUDA;
+      break;
+    }
   }
-  // the caller's stream continues after the last copies back
-  for (int sl = 0; sl < 2 && sl < groups; ++sl)
-    if (!ok(cudaStreamWaitEvent(cs, hp->out[sl], 0))) return ROLA_ERR_CUDA;
-  return ROLA_OK;
+  // whatever happened above, the caller's stream continues only after every
+  // copy this call enqueued (on success the last ones are the copies back)
+  const bool joined = ok(cudaEventRecord(hp->in[0], hp->h2d)) &&
+                      ok(cudaStreamWaitEvent(cs, hp->in[0], 0)) &&
+                      ok(cudaEventRecord(hp->out[0], hp->d2h)) &&
+                      ok(cudaStreamWaitEvent(cs, hp->out[0], 0));
+  return result != ROLA_OK ? result : (joined ? ROLA_OK : ROLA_ERR_CUDA);
 }
