@@ -103,3 +103,22 @@ def test_timed_layer_event_count_checked_on_host(lib):
     ev = (ctypes.c_void_p * 4)(4096, 4096, 4096, 4096)
     st = lib.rola_layer_fwd_timed(ctypes.byref(cs), ok, ok, ok, ok, ok, ok, None, ok, 1 << 30, None, None, ev, 4)
     assert st == 1  # ROLA_ERR_INVALID_ARG: three or five events
+
+
+@pytest.mark.parametrize("H,d,r,block,T,Hg,W,kb", [
+    (40, 128, 32, 128, 21, 45, 80, 18),   # 5 groups of 8 heads
+    (12, 128, 32, 128, 21, 30, 52, 26),   # 8 + 4 heads
+    (2, 64, 16, 64, 4, 16, 16, 4),        # one group of 2 heads (d = 64 groups hold 16)
+])
+def test_host_workspace_is_two_group_slots(lib, H, d, r, block, T, Hg, W, kb):
+    """The host-buffer layer stages P and gate of all heads, two slots of
+    q, k, v, out for one head group (2 KB of each token row), and the layer
+    workspace of one group."""
+    r256 = lambda n: -(-n // 256) * 256
+    s = rb.Shape(1, H, d, T, Hg, W, block, kb, r)
+    hc = min(H, -(-2048 // (2 * d)))
+    g = rb.Shape(1, hc, d, T, Hg, W, block, kb, r)
+    act = r256(s.N * hc * d * 2)
+    want = (r256(H * d * r * 2) + r256(H * 4) + 8 * act
+            + lib.rola_layer_workspace_bytes(ctypes.byref(g.c())))
+    assert lib.rola_layer_host_workspace_bytes(ctypes.byref(s.c())) == want
