@@ -90,8 +90,14 @@ int32_t rola_kb_from_sparsity(int32_t n_blocks, int32_t sparsity_permille);
 
 /* ---------------------------------------------------------------- selector */
 
-/* Workspace rola_select_blocks needs: 256-byte aligned, contents scratch. */
+/* Workspace rola_select_blocks needs: 256-byte aligned, contents scratch.
+ * 0 for an invalid shape. */
 size_t rola_select_workspace_bytes(const rola_shape_t* shape);
+
+/* The same number under the generic name: rola_select_blocks is the only one
+ * of the three hot-path steps (select, states, attention) that takes a
+ * workspace. */
+size_t rola_workspace_bytes(const rola_shape_t* shape);
 
 /* Block selector (write-up section 05: keep the high-energy query-key block
  * interactions).  For every (b, h): mean-pool q and k over each block's valid

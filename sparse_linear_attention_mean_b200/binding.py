@@ -22,7 +22,7 @@ DEVERR_TIMEOUT = 0x2
 
 EXPORTS = [
     "rola_status_string", "rola_num_blocks", "rola_kb_from_sparsity",
-    "rola_select_workspace_bytes", "rola_select_blocks", "rola_select_blocks_noalloc",
+    "rola_select_workspace_bytes", "rola_workspace_bytes", "rola_select_blocks", "rola_select_blocks_noalloc",
     "rola_block_states",
     "rola_attention_fwd", "rola_layer_workspace_bytes", "rola_layer_fwd", "rola_layer_fwd_timed",
     "rola_layer_kernel_launches",
@@ -90,7 +90,7 @@ def lib() -> ctypes.CDLL:
         L.rola_num_blocks.argtypes = [sp]
         L.rola_kb_from_sparsity.restype = i32
         L.rola_kb_from_sparsity.argtypes = [i32, i32]
-        for nm in ("rola_select_workspace_bytes", "rola_layer_workspace_bytes",
+        for nm in ("rola_select_workspace_bytes", "rola_workspace_bytes", "rola_layer_workspace_bytes",
                    "rola_layer_host_workspace_bytes"):
             getattr(L, nm).restype = sz
             getattr(L, nm).argtypes = [sp]

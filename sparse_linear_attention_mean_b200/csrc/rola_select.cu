@@ -339,6 +339,8 @@ extern "C" size_t rola_select_workspace_bytes(const rola_shape_t* s) {
   return rola_internal::round_up(pooled, 256) + rola_internal::round_up(scores, 256);
 }
 
+extern "C" size_t rola_workspace_bytes(const rola_shape_t* s) { return rola_select_workspace_bytes(s); }
+
 extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_t* q,
                                             const uint16_t* k, int32_t* idx, double* scores_opt,
                                             void* ws, size_t ws_bytes, void* stream) {

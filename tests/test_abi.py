@@ -49,8 +49,13 @@ def test_num_blocks_and_workspace_sizes(lib):
     assert rb.num_blocks(s) == 591
     cs = s.c()
     assert lib.rola_layer_workspace_bytes(ctypes.byref(cs)) > lib.rola_select_workspace_bytes(ctypes.byref(cs)) > 0
+    assert lib.rola_workspace_bytes(ctypes.byref(cs)) == lib.rola_select_workspace_bytes(ctypes.byref(cs))
+    # pooled q and k means and the scores, float64, each rounded up to 256 bytes
+    r256 = lambda n: -(-n // 256) * 256
+    assert lib.rola_select_workspace_bytes(ctypes.byref(cs)) == r256(2 * 40 * 591 * 128 * 8) + r256(40 * 591 * 591 * 8)
     bad = rb.Shape(1, 40, 128, 21, 45, 80, 128, 592, 32).c()   # k_b > n_blocks
     assert lib.rola_layer_workspace_bytes(ctypes.byref(bad)) == 0
+    assert lib.rola_workspace_bytes(ctypes.byref(bad)) == 0
 
 
 @pytest.mark.parametrize("field,value,status", [
