@@ -134,3 +134,43 @@ def rola_head_backward(q, k, v, P_h, g_h: float, dO, *, bs: int, idx, grid,
         G.dP += k[lo:hi].T @ duk
     G.dS_blk, G.dz_blk = dS_blk, dz_blk
     return G
+
+
+def transposed_mask(idx, nb: int):
+    """For each key block j, the ascending query blocks a whose kept list holds
+    j, in compressed form: ``rows[offsets[j]:offsets[j+1]]``.  The key-major
+    side of the backward walks these lists."""
+    idx = np.asarray(idx, dtype=np.int64)
+    lists = [[] for _ in range(nb)]
+    for a in range(idx.shape[0]):
+        for j in sorted(set(idx[a].tolist())):
+            lists[j].append(a)
+    offsets = np.zeros(nb + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum([len(x) for x in lists])
+    rows = np.array([a for x in lists for a in x], dtype=np.int32)
+    return offsets, rows
+
+
+def forward_stats(q, k, v, P_h, *, bs: int, idx, grid, rope_base: float = 10000.0):
+    """Per-row quantities a forward saves for the backward: the natural-log
+    log-sum-exp of the scaled scores over the kept keys, and the linear
+    branch's denominator psi_q . z_U (NaN for query blocks whose complement is
+    empty, where the linear branch is zero)."""
+    N, d = q.shape
+    nb = -(-N // bs)
+    T, Hg, W = grid
+    idx = np.asarray(idx, dtype=np.int64)
+    theta = rope_angles(N, T, Hg, W, P_h.shape[1], rope_base)
+    S_blk, z_blk, S, z = block_states(k, v, P_h, theta, bs)
+    lse = np.empty(N)
+    den = np.full(N, np.nan)
+    for a in range(nb):
+        lo, hi = block_range(a, bs, N)
+        J = kept_tokens(idx[a], bs, N)
+        s = (q[lo:hi] @ k[J].T) / math.sqrt(d)
+        m = s.max(axis=1)
+        lse[lo:hi] = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        if len(set(idx[a].tolist())) < nb:
+            _, z_U = complement_state(S_blk, z_blk, S, z, idx[a])
+            den[lo:hi] = phi(q[lo:hi] @ P_h) @ z_U
+    return lse, den

@@ -115,3 +115,44 @@ def test_a_planted_mistake_is_caught(monkeypatch):
     direction = rng.standard_normal(c["q"].shape)
     fd = _directional_fd(c, "q", direction)
     assert abs(fd - float((G.dq * direction).sum())) > 1e-4 * max(1.0, abs(fd))
+
+
+def test_transposed_mask_lists_every_keeping_query_block():
+    idx = np.array([[0, 2], [1, 2], [0, 3], [2, 3]])
+    offsets, rows = rbo.transposed_mask(idx, 4)
+    got = [rows[offsets[j]:offsets[j + 1]].tolist() for j in range(4)]
+    assert got == [[0, 2], [1], [0, 1, 3], [2, 3]]
+    # on a random mask: membership both ways, ascending, total = nb * k_b
+    rng = np.random.default_rng(9)
+    nb, kb = 37, 5
+    idx = np.stack([np.sort(rng.choice(nb, size=kb, replace=False)) for _ in range(nb)])
+    offsets, rows = rbo.transposed_mask(idx, nb)
+    assert offsets[-1] == nb * kb
+    for j in range(nb):
+        lst = rows[offsets[j]:offsets[j + 1]]
+        assert np.all(np.diff(lst) > 0)
+        assert set(lst.tolist()) == {a for a in range(nb) if j in idx[a]}
+
+
+def test_forward_stats_against_library_logsumexp():
+    from scipy.special import logsumexp
+    c = _case(8, 2)
+    lse, den = rbo.forward_stats(c["q"], c["k"], c["v"], c["P"], bs=BS, idx=c["idx"], grid=GRID)
+    N = c["q"].shape[0]
+    for a in range(c["idx"].shape[0]):
+        lo, hi = ro.block_range(a, BS, N)
+        J = ro.kept_tokens(c["idx"][a], BS, N)
+        s = c["q"][lo:hi] @ c["k"][J].T / np.sqrt(D)
+        assert np.allclose(lse[lo:hi], logsumexp(s, axis=1), rtol=0, atol=1e-12)
+    assert np.all(den > 0)
+    # the saved statistics reproduce the forward: o_sp = exp(s - lse) v, o_lin = num / den
+    res = ro.rola_head(c["q"], c["k"], c["v"], c["P"], c["g"], bs=BS, k_b=2, grid=GRID,
+                       rope_base=10000.0, idx=c["idx"])
+    for a, o_sp in res.o_sp.items():
+        lo, hi = ro.block_range(a, BS, N)
+        J = ro.kept_tokens(c["idx"][a], BS, N)
+        p = np.exp(c["q"][lo:hi] @ c["k"][J].T / np.sqrt(D) - lse[lo:hi, None])
+        assert np.allclose(p @ c["v"][J], o_sp, rtol=1e-12, atol=1e-12)
+    _, dense = rbo.forward_stats(c["q"], c["k"], c["v"], c["P"], bs=BS,
+                                 idx=np.tile(np.arange(4), (4, 1)), grid=GRID)
+    assert np.all(np.isnan(dense))
