@@ -34,7 +34,10 @@ the forward's steps in reverse order:
 Parity pins (tests/test_oracle_rola_backward.py): central finite differences of
 the forward oracle along random directions for every input; the dense limit
 (every block kept) against library autograd of scaled dot-product attention;
-the gate-zero case against library autograd of masked attention.
+the gate-zero case against library autograd of masked attention; a planted
+slip that the finite differences catch.  ``transposed_mask`` is checked by
+membership both ways, ``forward_stats`` against the library log-sum-exp and by
+rebuilding the forward's sparse output from it.
 """
 from __future__ import annotations
 
