@@ -127,3 +127,12 @@ def test_host_workspace_is_two_group_slots(lib, H, d, r, block, T, Hg, W, kb):
     want = (r256(H * d * r * 2) + r256(H * 4) + 8 * act
             + lib.rola_layer_workspace_bytes(ctypes.byref(g.c())))
     assert lib.rola_layer_host_workspace_bytes(ctypes.byref(s.c())) == want
+
+
+def test_binding_constants_match_the_header():
+    text = open(HEADER).read()
+    enum = dict((int(v), n) for n, v in re.findall(r"\b(ROLA_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
+    assert sorted(enum) == sorted(rb.STATUS)
+    defines = dict(re.findall(r"#define\s+ROLA_DEVERR_(\w+)\s+(0x[0-9a-fA-F]+)", text))
+    assert int(defines["BAD_INDEX"], 16) == rb.DEVERR_BAD_INDEX
+    assert int(defines["TIMEOUT"], 16) == rb.DEVERR_TIMEOUT
