@@ -1,7 +1,8 @@
 """The staged form of the RoLA gradient that a kernel implementation follows,
-checked against the gradient oracle: a query-major pass that recomputes the
-softmax from the saved per-row log-sum-exp and forms dQ, D = dO . o_sp and the
-query side of the linear branch (dS_U, dz_U per query block); the transposed
+checked against the gradient oracle: a query-major pass that forms the query
+side of the linear branch (dS_U, dz_U per query block, and o_lin again), D =
+dO . o - g dO . o_lin from the layer output, the softmax from the saved per-row
+log-sum-exp, and dQ; the transposed
 block mask; per key block, dS_b = (sum of all dS_U) - (those of the query blocks
 that keep b), the mirror of the forward's global-minus-kept states; and a
 key-major pass over the keeping query blocks for dK, dV and the key side of
@@ -29,31 +30,35 @@ def staged_backward(q, k, v, P, g, dO, bs, idx, grid):
     D = np.zeros(N)
     dSU, dzU = {}, {}
 
-    # query-major pass: softmax from the saved log-sum-exp, D = dO . o_sp, dQ,
-    # and the query side of the linear branch
+    # the layer output, as the forward wrote it
+    res = ro.rola_head(q, k, v, P, g, bs=bs, k_b=idx.shape[1], grid=grid, rope_base=10000.0, idx=idx)
+
+    # query-major pass: the query side of the linear branch first (it recomputes
+    # o_lin), then D = dO . o - g dO . o_lin = dO . o_sp, the softmax from the
+    # saved log-sum-exp, and dQ
     for a in range(nb):
         lo, hi = ro.block_range(a, bs, N)
+        o_lin = np.zeros((hi - lo, d))
+        if not np.isnan(den[lo]):  # NaN: every block kept, no linear branch
+            S_U, z_U = ro.complement_state(S_blk, z_blk, S, z, idx[a])
+            u = q[lo:hi] @ P
+            psi = ro.phi(u)
+            rho = ro.rotate(psi, theta[lo:hi])
+            o_lin = rho @ S_U / den[lo:hi, None]
+            dg += (dO[lo:hi] * o_lin).sum()
+            dnum = g * dO[lo:hi] / den[lo:hi, None]
+            dden = -(g * dO[lo:hi] * o_lin).sum(1) / den[lo:hi]
+            dpsi = dden[:, None] * z_U + ro.rotate(dnum @ S_U.T, -theta[lo:hi])
+            du = dpsi * rbo.phi_grad(u)
+            dq[lo:hi] += du @ P.T
+            dP += q[lo:hi].T @ du
+            dSU[a] = rho.T @ dnum
+            dzU[a] = (dden[:, None] * psi).sum(0)
+        D[lo:hi] = (dO[lo:hi] * res.o[a]).sum(1) - g * (dO[lo:hi] * o_lin).sum(1)
         J = ro.kept_tokens(idx[a], bs, N)
         p = np.exp(q[lo:hi] @ k[J].T * sc - lse[lo:hi, None])
-        D[lo:hi] = (dO[lo:hi] * (p @ v[J])).sum(1)
         ds = p * (dO[lo:hi] @ v[J].T - D[lo:hi, None])
         dq[lo:hi] += ds @ k[J] * sc
-        if np.isnan(den[lo]):
-            continue  # every block kept: no linear branch
-        S_U, z_U = ro.complement_state(S_blk, z_blk, S, z, idx[a])
-        u = q[lo:hi] @ P
-        psi = ro.phi(u)
-        rho = ro.rotate(psi, theta[lo:hi])
-        o_lin = rho @ S_U / den[lo:hi, None]
-        dg += (dO[lo:hi] * o_lin).sum()
-        dnum = g * dO[lo:hi] / den[lo:hi, None]
-        dden = -(g * dO[lo:hi] * o_lin).sum(1) / den[lo:hi]
-        dpsi = dden[:, None] * z_U + ro.rotate(dnum @ S_U.T, -theta[lo:hi])
-        du = dpsi * rbo.phi_grad(u)
-        dq[lo:hi] += du @ P.T
-        dP += q[lo:hi].T @ du
-        dSU[a] = rho.T @ dnum
-        dzU[a] = (dden[:, None] * psi).sum(0)
 
     # block-state gradients: all query blocks' dS_U minus those that keep the block
     off, rows = rbo.transposed_mask(idx, nb)
