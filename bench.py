@@ -229,7 +229,7 @@ def run_gpu(args) -> int:
     gate = torch.from_numpy(inp["gate"]).cuda()
     stream = torch.cuda.current_stream()
 
-    # the layer's own entry point; three events split it into its two stages
+    # the layer's own entry point
     layer = rb.Layer(shape)
     out = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device="cuda")
     # five events: the q/k/v pass (block means + states), scores + top-k,
@@ -320,7 +320,9 @@ def run_gpu(args) -> int:
             "gpu_launches": K * launches_per_step,
             "clocks": clk.summary(),
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:
+            # the host-core oracle is timed at one GPU only (the multi-GPU
+            # lines keep the other ranks waiting as little as possible)
             line["cpu_baseline"] = cpu_baseline(w, inp)
         print(json.dumps(line))
     if world > 1:
