@@ -264,6 +264,22 @@ def run_gpu(args) -> int:
     flop = w.sparse_flops()
     value = job_tflops(flop, K, world, total_ms)
 
+    # the same layer with the mask of an earlier step reused (cross-step
+    # pattern reuse: no selection kernels; block states and attention as usual)
+    idx_keep = torch.empty((w.B, w.H, w.n_blocks, w.k_b), dtype=torch.int32, device="cuda")
+    layer.run_ex(q, k, v, P, gate, idx_keep, out=out, stream=stream)
+    for _ in range(args.warmup):
+        layer.run_ex(q, k, v, P, gate, idx_keep, reuse_mask=True, out=out, stream=stream)
+    torch.cuda.synchronize()
+    ev_r = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for s_ in range(K):
+        layer.run_ex(q, k, v, P, gate, idx_keep, reuse_mask=True, out=out, stream=stream, events=ev_r[s_])
+    torch.cuda.synchronize()
+    assert int(layer.dev_err.item()) == 0
+    reuse_ms = statistics.mean(e[0].elapsed_time(e[4]) for e in ev_r)
+    reuse = {"ms_per_layer": reuse_ms, "tflops": flop / (reuse_ms * 1e-3) / 1e12,
+             "selection_skipped_ms": statistics.mean(per_stage["score+topk"]) if "score+topk" in per_stage else None}
+
     # one FP8 W8A8 projection of the full attention block (x [N, 5120] ->
     # [N, 5120]: quantisation + tcgen05 GEMM), timed on its own after the layer
     fp8 = None
@@ -317,9 +333,15 @@ def run_gpu(args) -> int:
                          "peak_source": peaks["source"] + " bf16 burst"},
             "e2e": e2e,
             "fp8_projection": fp8,
+            "mask_reuse": reuse,
             "gpu_launches": K * launches_per_step,
             "clocks": clk.summary(),
         }
+        if args.per_config and world == 1:
+            flush = L2Flush()
+            line["per_config"] = {str(i): config_report(i, stream, peaks, flush, 10, 50)
+                                  for i in (0, 1, 2, 3)}
+            line["per_config"]["4"] = block_report(stream, peaks, flush, 3, 10)
         if not args.no_cpu_baseline and world == 1:
             # the host-core oracle is timed at one GPU only (the multi-GPU
             # lines keep the other ranks waiting as little as possible)
@@ -344,6 +366,199 @@ def hbm_report(w, stage_ms: dict, peaks: dict) -> dict:
             gbs = nbytes / (stage_ms[nm] * 1e-3) / 1e9
             out[nm] = {"bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
     return out
+
+
+# ---------------------------------------------------------------- per-config report
+
+def _pct(xs, q):
+    return float(np.percentile(np.asarray(xs, dtype=np.float64), q))
+
+
+class L2Flush:
+    """Writes a 256 MB buffer (twice the 126 MB L2) so that a timed rep starts
+    with nothing of its inputs in L2."""
+
+    def __init__(self):
+        import torch
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def __call__(self, stream):
+        import torch
+        with torch.cuda.stream(stream):
+            self.buf.fill_(1)
+
+
+def _timed_reps(fn, stream, flush, warmup: int, reps: int, n_events: int = 2):
+    """Runs fn(events) warmup + reps times with an L2 flush before each rep;
+    returns the per-rep lists of the intervals between consecutive events."""
+    import torch
+    for _ in range(warmup):
+        flush(stream)
+        fn([torch.cuda.Event(enable_timing=True) for _ in range(n_events)])
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(reps):
+        flush(stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+        fn(ev)
+        evs.append(ev)
+    torch.cuda.synchronize()
+    return [[ev[i].elapsed_time(ev[i + 1]) for i in range(n_events - 1)] for ev in evs]
+
+
+def config_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
+    """One attention workload through the layer entry point: ms per layer and
+    per stage (p50 / p95), effective TFLOP/s of the layer and of the attention
+    kernel against the bf16 peak, HBM rate of the pass over q, k, v and of the
+    state totals, and the mask against the oracle's selection (mismatching rows
+    outside near-ties, near-tie rows)."""
+    import torch
+    from oracle import rola_oracle as ro
+    from sparse_linear_attention_mean_b200 import binding as rb
+    from sparse_linear_attention_mean_b200 import synth
+    w = synth.WORKLOADS[wid]
+    shape = rb.Shape.of(w)
+    inp = synth.make_inputs(w)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+    q, k, v, P = dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["P"])
+    gate = torch.from_numpy(inp["gate"]).cuda()
+    layer = rb.Layer(shape)
+    out = torch.empty_like(q)
+    idx = torch.empty((w.B, w.H, w.n_blocks, w.k_b), dtype=torch.int32, device="cuda")
+    fused = rb.layer_launches(shape) == 5
+    n_ev = 5 if fused else 3
+    per = _timed_reps(lambda ev: layer(q, k, v, P, gate, out=out, idx_out=idx, stream=stream, events=ev),
+                      stream, flush, warmup, reps, n_ev)
+    assert int(layer.dev_err.item()) == 0
+    layer_ms = [sum(x) for x in per]
+    att_ms = [x[-1] for x in per]
+    flop = w.sparse_flops()
+    rep = {"workload": w.name, "H": w.H, "d": w.d, "grid_thw": [w.T, w.Hg, w.W], "block": w.block,
+           "n_blocks": w.n_blocks, "k_b": w.k_b, "rank": w.r, "flop": flop, "reps": reps, "warmup": warmup,
+           "l2": "256 MB flush before each rep",
+           "layer_ms_p50": _pct(layer_ms, 50), "layer_ms_p95": _pct(layer_ms, 95),
+           "attention_ms_p50": _pct(att_ms, 50), "attention_ms_p95": _pct(att_ms, 95)}
+    rep["layer_tflops"] = flop / (rep["layer_ms_p50"] * 1e-3) / 1e12
+    rep["attention_tflops"] = flop / (rep["attention_ms_p50"] * 1e-3) / 1e12
+    rep["layer_frac_of_bf16_peak"] = rep["layer_tflops"] / peaks["bf16_tflops"]
+    rep["attention_frac_of_bf16_peak"] = rep["attention_tflops"] / peaks["bf16_tflops"]
+    if fused:
+        names = ("prep", "score+topk", "state_totals", "attention")
+        rep["stages_ms_p50"] = {nm: _pct([x[i] for x in per], 50) for i, nm in enumerate(names)}
+        rep["hbm"] = hbm_report(w, rep["stages_ms_p50"], peaks)
+    else:
+        rep["stages_ms_p50"] = {"select+states": _pct([x[0] for x in per], 50),
+                                "attention": _pct([x[1] for x in per], 50)}
+    idx_ref, sig = ro.select_all(inp, w.block, w.k_b)
+    got = idx.cpu().numpy()
+    ties = bad = n_tie_rows = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            tie_rows = set(ro.near_ties(sig[b, h], w.k_b))
+            n_tie_rows += len(tie_rows)
+            for a in np.nonzero((got[b, h] != idx_ref[b, h]).any(axis=1))[0]:
+                if int(a) in tie_rows:
+                    ties += 1
+                else:
+                    bad += 1
+    rep["mask"] = {"rows": int(w.B * w.H * w.n_blocks), "mismatch_outside_near_ties": bad,
+                   "near_tie_rows": n_tie_rows, "differing_near_tie_rows": ties}
+    del q, k, v, out, layer
+    torch.cuda.empty_cache()
+    return rep
+
+
+def block_report(stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
+    """The full 14B-720P attention block (x [75600, 5120]): per-token
+    quantisation + the Q, K, V W8A8 projections, the RoLA layer, quantisation
+    + the output projection; and the block's FFN (5120 -> 13824 -> 5120, W8A8,
+    GELU).  ms p50 / p95 per part, the GEMMs' effective TFLOP/s against the
+    FP8 peak (2 x the measured bf16 peak, the nominal ratio)."""
+    import torch
+    from sparse_linear_attention_mean_b200 import binding as rb
+    from sparse_linear_attention_mean_b200 import synth
+    w = synth.WORKLOADS[4]
+    inp = synth.make_block_inputs(w)
+    M, D = w.B * w.N, w.model_dim
+    x = torch.from_numpy(np.ascontiguousarray(inp["x"])).view(torch.bfloat16).cuda()
+    wts = {nm: rb.fp8_quantize_weight(torch.from_numpy(np.ascontiguousarray(inp[nm])).cuda())
+           for nm in ("Wq", "Wk", "Wv", "Wo")}
+    P = torch.from_numpy(np.ascontiguousarray(inp["P"])).view(torch.bfloat16).cuda()
+    gate = torch.from_numpy(inp["gate"]).cuda()
+    shape = rb.Shape.of(w)
+    layer = rb.Layer(shape)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qkv = {nm: torch.empty((M, D), dtype=torch.bfloat16, device="cuda") for nm in ("Wq", "Wk", "Wv")}
+    o = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+    xq = torch.empty((M, D), dtype=torch.uint8, device="cuda")
+    xs = torch.empty((M,), dtype=torch.float32, device="cuda")
+    lib = rb.lib()
+    import ctypes
+    P_ = lambda t: ctypes.c_void_p(t.data_ptr())
+    cs = ctypes.c_void_p(stream.cuda_stream)
+
+    def quant(src):
+        assert lib.fp8_quantize_rows_bf16(M, D, P_(src), P_(xq), P_(xs), cs) == 0
+
+    def gemm(wq, ws, dst):
+        assert lib.fp8_gemm_w8a8(M, D, D, P_(xq), P_(xs), P_(wq), P_(ws), P_(dst), P_(err), cs) == 0
+
+    def step(ev):
+        ev[0].record(stream)
+        quant(x)
+        for nm in ("Wq", "Wk", "Wv"):
+            gemm(*wts[nm], qkv[nm])
+        ev[1].record(stream)
+        layer(qkv["Wq"].view(w.B, w.N, w.H, w.d), qkv["Wk"].view(w.B, w.N, w.H, w.d),
+              qkv["Wv"].view(w.B, w.N, w.H, w.d), P, gate, out=o.view(w.B, w.N, w.H, w.d), stream=stream)
+        ev[2].record(stream)
+        quant(o)
+        gemm(*wts["Wo"], y)
+        ev[3].record(stream)
+
+    per = _timed_reps(step, stream, flush, warmup, reps, 4)
+    assert int(err.item()) == 0 and int(layer.dev_err.item()) == 0
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    gflop = 2.0 * M * D * D
+    names = ("quant+qkv_gemms", "rola_layer", "quant+out_gemm")
+    rep = {"workload": w.name, "reps": reps, "warmup": warmup, "l2": "256 MB flush before each rep",
+           "fp8_peak_tflops": fp8_peak,
+           "fp8_peak_source": peaks["source"] + " bf16 burst x 2 (nominal fp8:bf16 ratio)"}
+    for i, nm in enumerate(names):
+        rep[nm + "_ms_p50"] = _pct([x[i] for x in per], 50)
+        rep[nm + "_ms_p95"] = _pct([x[i] for x in per], 95)
+    tot = [sum(x) for x in per]
+    rep["block_ms_p50"], rep["block_ms_p95"] = _pct(tot, 50), _pct(tot, 95)
+    rep["qkv_tflops"] = 3 * gflop / (rep["quant+qkv_gemms_ms_p50"] * 1e-3) / 1e12
+    rep["qkv_frac_of_fp8_peak"] = rep["qkv_tflops"] / fp8_peak
+    rep["out_tflops"] = gflop / (rep["quant+out_gemm_ms_p50"] * 1e-3) / 1e12
+    rep["out_frac_of_fp8_peak"] = rep["out_tflops"] / fp8_peak
+    del qkv, o, layer
+    torch.cuda.empty_cache()
+    # the block's FFN
+    ffw = synth.make_ffn_weights(w)
+    F = ffw["W1"].shape[0]
+    w1q, w1s = rb.fp8_quantize_weight(torch.from_numpy(ffw["W1"]).cuda())
+    w2q, w2s = rb.fp8_quantize_weight(torch.from_numpy(ffw["W2"]).cuda())
+    ws_ffn = torch.empty(lib.fp8_ffn_workspace_bytes(M, D, F), dtype=torch.uint8, device="cuda")
+
+    def ffn(ev):
+        ev[0].record(stream)
+        rb.fp8_ffn(x, w1q, w1s, w2q, w2s, out=y, workspace=ws_ffn, dev_err=err, stream=stream)
+        ev[1].record(stream)
+
+    per = _timed_reps(ffn, stream, flush, max(1, warmup // 2), max(3, reps // 3), 2)
+    assert int(err.item()) == 0
+    ffn_ms = [x[0] for x in per]
+    ffn_flop = 2 * 2.0 * M * D * F
+    rep["ffn"] = {"shape_m_d_f": [M, D, F], "activation": "gelu_tanh",
+                  "ms_p50": _pct(ffn_ms, 50), "ms_p95": _pct(ffn_ms, 95),
+                  "tflops": ffn_flop / (_pct(ffn_ms, 50) * 1e-3) / 1e12}
+    rep["ffn"]["frac_of_fp8_peak"] = rep["ffn"]["tflops"] / fp8_peak
+    del ws_ffn
+    torch.cuda.empty_cache()
+    return rep
 
 
 def fp8_projection(M: int, D: int, stream, reps: int = 5) -> dict:
@@ -411,6 +626,9 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass (profiling runs)")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 projection timing")
+    ap.add_argument("--per-config", dest="per_config", action="store_true", default=True,
+                    help="add the per-workload report (default at one GPU)")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false")
     ap.add_argument("--fp8-only", action="store_true",
                     help="time only the FP8 projection (x [rows, 5120] -> [rows, 5120]); profiling captures")
     ap.add_argument("--fp8-rows", type=int, default=75600, help="rows of x for --fp8-only")

@@ -119,8 +119,10 @@ rola_status_t rola_select_blocks(const rola_shape_t* shape, const uint16_t* q, c
  * it exists for callers that cannot provide device memory at the call site).
  * Same inputs, output and results as rola_select_blocks (no scores output).
  * ROLA_ERR_WORKSPACE when rola_select_workspace_bytes(shape) exceeds 16 MiB.
- * The first call on a device looks up the array's address (set-up work: make
- * it before any stream capture).  Nothing is allocated and nothing needs
+ * Every call looks up the array's device address on the current device, so
+ * the entry point stays valid across a device reset; the first call on a
+ * device also loads the library's device code there (set-up work: make it
+ * before any stream capture).  Nothing is allocated and nothing needs
  * clearing; calls that overlap in time on one device share the array and
  * race, so callers serialise them. */
 rola_status_t rola_select_blocks_noalloc(const rola_shape_t* shape, const uint16_t* q,
@@ -179,6 +181,72 @@ rola_status_t rola_attention_fwd(const rola_shape_t* shape, const uint16_t* q, c
                                  const float* z_glb, const float* gate, uint16_t* out,
                                  int32_t* dev_err, void* stream);
 
+/* rola_attention_fwd with the bound on each of the kernel's pipeline waits
+ * given in nanoseconds (rola_attention_fwd uses 1 s).  The pages describe no
+ * such call: it is this library's failure detection.  A wait that runs out
+ * makes its CTA stop, wait (at most 1 s each) for the copies and MMAs it has
+ * in flight, free its tensor memory and return; the launch's later CTAs skip
+ * their work, ROLA_DEVERR_TIMEOUT is ORed into *dev_err and `out` is
+ * incomplete.  The device stays usable: later calls run normally.
+ * wait_limit_ns = 0 makes a wait give up as soon as it finds its stage not
+ * ready yet, so a test can run the timeout path without any fault.  Other
+ * arguments, results and errors as rola_attention_fwd. */
+rola_status_t rola_attention_fwd_bounded(const rola_shape_t* shape, const uint16_t* q,
+                                         const uint16_t* k, const uint16_t* v, const int32_t* idx,
+                                         const uint16_t* P, const float* S_blk, const float* z_blk,
+                                         const float* S_glb, const float* z_glb, const float* gate,
+                                         uint16_t* out, int32_t* dev_err, uint64_t wait_limit_ns,
+                                         void* stream);
+
+/* ---------------------------------------------------------------- backward */
+
+/* rola_attention_fwd (d = 128, 128-token blocks, k_b <= 256, n_blocks <= 1024)
+ * that also saves, per row, what rola_attention_bwd reads:
+ *   lse  float [B, H, N]: natural log of sum over the kept valid keys of
+ *        exp(q . k / sqrt(d)) (-inf for a row without kept blocks);
+ *   den  float [B, H, N]: the linear branch's denominator psi_q . z_U (NaN
+ *        when the complement is empty).
+ * Other arguments, results and errors as rola_attention_fwd; other shapes:
+ * ROLA_ERR_UNSUPPORTED.  S_blk and S_glb 32-byte aligned, P 16-byte. */
+rola_status_t rola_attention_fwd_train(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
+                                       const uint16_t* v, const int32_t* idx, const uint16_t* P,
+                                       const float* S_blk, const float* z_blk, const float* S_glb,
+                                       const float* z_glb, const float* gate, uint16_t* out, float* lse,
+                                       float* den, int32_t* dev_err, void* stream);
+
+/* Workspace of rola_attention_bwd (256-byte aligned), 0 for an invalid or
+ * unsupported shape. */
+size_t rola_attention_bwd_workspace_bytes(const rola_shape_t* shape);
+
+/* Gradients of sum(dout * out) for the forward above, the block mask held
+ * fixed (selection passes no gradient).  The SparkDiffusion write-up (section
+ * 05) and project blog ("A simple staging principle", item 1) adapt the dense
+ * model to 97 % sparsity by a short sparse warm-up that trains through RoLA;
+ * the pages print no backward, so the gradient is the chain rule through the
+ * forward's steps in reverse: the sparse branch from the saved log-sum-exp
+ * (P = exp(S / sqrt(d) - lse), D = dout . o_sp), the linear branch through
+ * o_lin = rho_q^T S_U / (psi_q . z_U), the complement S_U = S - sum_kept S_b,
+ * the block states S_b = sum rho_k v^T, z_b = sum psi_k, the rotary
+ * rotation, the feature map elu + 1 and the projection P_h.
+ *   q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate: the forward's inputs
+ *   out, lse, den: its output and saved statistics (rola_attention_fwd_train)
+ *   dout   bf16 [B, N, H, d], the gradient reaching out
+ *   dq, dk, dv  out, bf16 [B, N, H, d] (padding rows not written)
+ *   dP     out, float [H, d, r];   dgate  out, float [H]
+ * Two passes, no atomics (deterministic): a query-major pass (dq, the query
+ * side of the linear branch, D) and a key-major pass over the query blocks
+ * that keep each key block (dk, dv, the key side); contractions on the
+ * tensor cores (tcgen05).  Supported: d = 128, 128-token blocks, r 16 or 32,
+ * k_b <= 256, n_blocks <= 1024 (else ROLA_ERR_UNSUPPORTED).  16-byte aligned
+ * activations and gradients; dev_err as in rola_attention_fwd. */
+rola_status_t rola_attention_bwd(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
+                                 const uint16_t* v, const int32_t* idx, const uint16_t* P,
+                                 const float* S_blk, const float* z_blk, const float* S_glb,
+                                 const float* z_glb, const float* gate, const uint16_t* out,
+                                 const float* lse, const float* den, const uint16_t* dout, uint16_t* dq,
+                                 uint16_t* dk, uint16_t* dv, float* dP, float* dgate, void* ws,
+                                 size_t ws_bytes, int32_t* dev_err, void* stream);
+
 /* ---------------------------------------------------------------- whole layer */
 
 /* Workspace of rola_layer_fwd: selector scratch, idx and the states. */
@@ -213,6 +281,38 @@ rola_status_t rola_layer_fwd_timed(const rola_shape_t* shape, const uint16_t* q,
                                    uint16_t* out, int32_t* idx_out, void* ws, size_t ws_bytes,
                                    int32_t* dev_err, void* stream, void* const* events,
                                    int32_t n_events);
+
+/* Options of rola_layer_fwd_ex. */
+typedef struct {
+  /* Per-head kept counts, device int32 [H] (each in 1..shape->k_b), or NULL
+   * for shape->k_b in every head.  The Video-Generation-101 chapter page on
+   * sparse attention lists head-adaptive block sparsity (AdaSpa) among the
+   * sparse-attention methods: heads differ in how concentrated their
+   * attention is, so each head may keep its own number of blocks.  idx rows
+   * keep the stride shape->k_b; a head keeping kb_h blocks fills the first
+   * kb_h entries of its rows (ascending) and the selector writes -1 into the
+   * rest.  A count outside 1..k_b is clamped into it and reported through
+   * ROLA_DEVERR_BAD_INDEX. */
+  const int32_t* kb_per_head;
+  /* 0: select the mask and (when idx_io is not NULL) write it to idx_io.
+   * Nonzero: idx_io holds the mask to use (for example the one selected at an
+   * earlier diffusion step: the same chapter page lists cross-step reuse of
+   * the sparsity pattern, RAPID); no selection kernel runs, the block states
+   * and the attention run as usual. */
+  int32_t reuse_mask;
+} rola_layer_opts_t;
+
+/* rola_layer_fwd_timed with options (opts may be NULL: then the call equals
+ * rola_layer_fwd_timed with idx_out = idx_io).  idx_io: int32 [B, H,
+ * n_blocks, k_b], an output unless opts->reuse_mask, then an input (required,
+ * rows validated by the attention kernel as in rola_attention_fwd).
+ * events / n_events as in rola_layer_fwd_timed (NULL / 0 for none); with a
+ * reused mask the scores-and-top-k interval is empty. */
+rola_status_t rola_layer_fwd_ex(const rola_shape_t* shape, const rola_layer_opts_t* opts,
+                                const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                const uint16_t* P, const float* gate, uint16_t* out,
+                                int32_t* idx_io, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                void* stream, void* const* events, int32_t n_events);
 
 /* Number of kernels one rola_layer_fwd call launches for `shape` (0 for an
  * invalid or unsupported shape); memory copies are not counted. */
@@ -272,6 +372,21 @@ rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
                             const float* x_scale, const uint8_t* w_q, const float* w_scale,
                             uint16_t* y, int32_t* dev_err, void* stream);
 
+/* Activation applied in the GEMM epilogue (fp8_gemm_w8a8_act). */
+#define ROLA_ACT_NONE 0
+#define ROLA_ACT_GELU_TANH 1 /* 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))) */
+
+/* fp8_gemm_w8a8 with an activation applied to the scaled fp32 product
+ * before the bf16 rounding: y = bf16(act(product * x_scale * w_scale)).
+ * GELU in its tanh form serves the FFN's up projection (write-up section 07:
+ * the FFN projections run in W8A8 FP8 too; the pages name no activation, so
+ * this library takes the tanh form).  act must be ROLA_ACT_NONE or
+ * ROLA_ACT_GELU_TANH, else ROLA_ERR_INVALID_ARG; other arguments as
+ * fp8_gemm_w8a8. */
+rola_status_t fp8_gemm_w8a8_act(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
+                                const float* x_scale, const uint8_t* w_q, const float* w_scale,
+                                int32_t act, uint16_t* y, int32_t* dev_err, void* stream);
+
 /* Workspace of fp8_linear_w8a8: the quantised activations and their scales. */
 size_t fp8_linear_workspace_bytes(int32_t M, int32_t K);
 
@@ -280,6 +395,25 @@ size_t fp8_linear_workspace_bytes(int32_t M, int32_t K);
 rola_status_t fp8_linear_w8a8(int32_t M, int32_t N, int32_t K, const uint16_t* x,
                               const uint8_t* w_q, const float* w_scale, uint16_t* y, void* ws,
                               size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Workspace of fp8_ffn_w8a8 (256-byte aligned): codes and scales of x, the
+ * bf16 hidden activation [M, F], and its codes and scales. */
+size_t fp8_ffn_workspace_bytes(int32_t M, int32_t D, int32_t F);
+
+/* The transformer block's FFN with both projections in W8A8 FP8 E4M3
+ * (write-up section 07: the FFN projections are quantised like the attention
+ * ones):  y = W2 gelu_tanh(W1 x)  for x bf16 [M, D], w1_q [F, D], w2_q [D, F]
+ * (E4M3 bytes, K-major) with per-output-channel scales w1_scale [F],
+ * w2_scale [D], and y bf16 [M, D].  Steps, in order: per-token quantisation of
+ * x; the up projection with GELU in its epilogue, written as bf16 [M, F] into
+ * the workspace; per-token quantisation of that hidden activation; the down
+ * projection.  D and F multiples of 32 (and of 16 for the quantisation), at
+ * most 16384.  Device pointers owned by the caller; ws of
+ * fp8_ffn_workspace_bytes(M, D, F) bytes; dev_err as in fp8_gemm_w8a8. */
+rola_status_t fp8_ffn_w8a8(int32_t M, int32_t D, int32_t F, const uint16_t* x,
+                           const uint8_t* w1_q, const float* w1_scale, const uint8_t* w2_q,
+                           const float* w2_scale, uint16_t* y, void* ws, size_t ws_bytes,
+                           int32_t* dev_err, void* stream);
 
 #ifdef __cplusplus
 }

@@ -17,6 +17,13 @@ per-token dynamic activation scales:
   by floating point, so both sides make that decision in float32;
 * ``y[m, n] = (sum_k dec(q_x[m, k]) dec(q_w[n, k])) * s_x[m] * s_w[n]``, in float64.
 
+The FFN of the transformer block (the write-up's "FFN projections", section 07)
+is ``y = W2 gelu(W1 x)`` with both projections in W8A8.  The pages fix neither
+the hidden width nor the activation; this library takes the tanh form of GELU
+and, for the 14B model, a hidden width of 13824 (see ``ffn_w8a8``).  The hidden
+activation is stored in bf16 between the two projections, as a GPU
+implementation keeps it.
+
 The E4M3 codec follows the OCP 8-bit floating point specification (OFP8):
 1 sign, 4 exponent (bias 7) and 3 mantissa bits; exponent field 0 is
 subnormal (m/8 * 2^-6); S.1111.111 is NaN; there is no infinity; the largest
@@ -24,6 +31,8 @@ finite magnitude is 1.75 * 2^8 = 448.  Conversion rounds to nearest, ties to
 even, and saturates to +-448 (the "satfinite" mode).
 """
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -92,3 +101,31 @@ def linear_w8a8(x_f32: np.ndarray, w_codes, w_scale) -> np.ndarray:
     """Activation quantisation followed by the scaled FP8 product."""
     xq, sx = quantize_rows(x_f32)
     return gemm_w8a8(xq, sx, w_codes, w_scale)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value (ties to even) of float64 values, as float64:
+    first to float32 (nearest), then the 16 low bits of the float32 pattern
+    rounded away to nearest even.  Finite inputs."""
+    u = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32)).view(np.uint32)
+    u = u.astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def gelu_tanh(u: np.ndarray) -> np.ndarray:
+    """GELU in its tanh form: 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)))."""
+    u = np.asarray(u, dtype=np.float64)
+    return 0.5 * u * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+
+
+def ffn_w8a8(x_f32: np.ndarray, w1_codes, w1_scale, w2_codes, w2_scale):
+    """The block's FFN with both projections in W8A8, in the order the method
+    applies the steps: per-token quantisation of x, the up projection
+    (hidden = W1 x), GELU, the hidden activation stored as bf16, per-token
+    quantisation of that activation, the down projection.  Returns
+    (h, y): h the bf16 hidden activation [M, F] as float64, y [M, D] float64."""
+    hidden = linear_w8a8(x_f32, w1_codes, w1_scale)
+    h = round_bf16(gelu_tanh(hidden))
+    y = linear_w8a8(h.astype(np.float32), w2_codes, w2_scale)
+    return h, y

@@ -289,17 +289,38 @@ def select_all(inputs: dict, bs: int, k_b: int):
 
 
 def rola_forward(inputs: dict, *, bs: int, k_b: int, grid, rope_base: float = 10000.0,
-                 idx=None, heads=None, qblocks=None):
-    """RoLA forward over (batch, head) pairs; returns {(b, h): HeadResult}."""
+                 idx=None, heads=None, qblocks=None, kb_per_head=None):
+    """RoLA forward over (batch, head) pairs; returns {(b, h): HeadResult}.
+    ``kb_per_head`` (length H): head h keeps kb_per_head[h] blocks, and a
+    given ``idx`` holds them in the first kb_per_head[h] entries of each row."""
     B, N, H, d = inputs["q"].shape
     out = {}
     for b in range(B):
         for h in (range(H) if heads is None else heads):
             q, k, v, P_h = head_slices(inputs, b, h)
-            out[(b, h)] = rola_head(q, k, v, P_h, float(inputs["gate"][h]), bs=bs, k_b=k_b,
+            kh = k_b if kb_per_head is None else int(kb_per_head[h])
+            out[(b, h)] = rola_head(q, k, v, P_h, float(inputs["gate"][h]), bs=bs, k_b=kh,
                                     grid=grid, rope_base=rope_base,
-                                    idx=None if idx is None else idx[b, h], qblocks=qblocks)
+                                    idx=None if idx is None else idx[b, h][:, :kh], qblocks=qblocks)
     return out
+
+
+def select_all_per_head(inputs: dict, bs: int, kb_per_head, k_b_max: int):
+    """Selector with a kept count per head (head-adaptive sparsity): head h
+    keeps its kb_per_head[h] best blocks per query block; rows have k_b_max
+    entries, the unused ones -1.  Returns idx [B, H, nb, k_b_max] and sigma."""
+    B, N, H, d = inputs["q"].shape
+    nb = -(-N // bs)
+    idx = np.full((B, H, nb, k_b_max), -1, dtype=np.int32)
+    sig = np.empty((B, H, nb, nb))
+    for b in range(B):
+        for h in range(H):
+            qb = pool_blocks(bf16_to_f64(inputs["q"][b, :, h, :]), bs)
+            kb = pool_blocks(bf16_to_f64(inputs["k"][b, :, h, :]), bs)
+            sig[b, h] = block_scores(qb, kb)
+            kh = int(kb_per_head[h])
+            idx[b, h, :, :kh] = select_topk(sig[b, h], kh)
+    return idx, sig
 
 
 def assemble_output(results: dict, B: int, N: int, H: int, d: int, bs: int) -> np.ndarray:

@@ -19,17 +19,24 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace"
           4: "CUDA error", 5: "alignment"}
 DEVERR_BAD_INDEX = 0x1
 DEVERR_TIMEOUT = 0x2
+ACT_NONE = 0
+ACT_GELU_TANH = 1
 
 EXPORTS = [
     "rola_status_string", "rola_num_blocks", "rola_kb_from_sparsity",
     "rola_select_workspace_bytes", "rola_workspace_bytes", "rola_select_blocks", "rola_select_blocks_noalloc",
     "rola_block_states",
-    "rola_attention_fwd", "rola_layer_workspace_bytes", "rola_layer_fwd", "rola_layer_fwd_timed",
-    "rola_layer_kernel_launches",
+    "rola_attention_fwd", "rola_attention_fwd_bounded", "rola_layer_workspace_bytes", "rola_layer_fwd", "rola_layer_fwd_timed",
+    "rola_layer_kernel_launches", "rola_layer_fwd_ex",
+    "rola_attention_fwd_train", "rola_attention_bwd_workspace_bytes", "rola_attention_bwd",
     "rola_layer_host_workspace_bytes", "rola_layer_fwd_host",
-    "fp8_quantize_rows_bf16", "fp8_quantize_weight", "fp8_gemm_w8a8",
-    "fp8_linear_workspace_bytes", "fp8_linear_w8a8",
+    "fp8_quantize_rows_bf16", "fp8_quantize_weight", "fp8_gemm_w8a8", "fp8_gemm_w8a8_act",
+    "fp8_linear_workspace_bytes", "fp8_linear_w8a8", "fp8_ffn_workspace_bytes", "fp8_ffn_w8a8",
 ]
+
+
+class LayerOpts(ctypes.Structure):
+    _fields_ = [("kb_per_head", ctypes.c_void_p), ("reuse_mask", ctypes.c_int32)]
 
 
 class RolaShape(ctypes.Structure):
@@ -102,11 +109,22 @@ def lib() -> ctypes.CDLL:
         L.rola_block_states.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.rola_attention_fwd.restype = ctypes.c_int
         L.rola_attention_fwd.argtypes = [sp] + [vp] * 12 + [vp]
+        L.rola_attention_fwd_bounded.restype = ctypes.c_int
+        L.rola_attention_fwd_bounded.argtypes = [sp] + [vp] * 12 + [ctypes.c_uint64, vp]
         L.rola_layer_fwd.restype = ctypes.c_int
         L.rola_layer_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         L.rola_layer_fwd_timed.restype = ctypes.c_int
         L.rola_layer_fwd_timed.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp,
                                            ctypes.POINTER(ctypes.c_void_p), i32]
+        L.rola_layer_fwd_ex.restype = ctypes.c_int
+        L.rola_layer_fwd_ex.argtypes = [sp, ctypes.POINTER(LayerOpts), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                        vp, ctypes.POINTER(ctypes.c_void_p), i32]
+        L.rola_attention_fwd_train.restype = ctypes.c_int
+        L.rola_attention_fwd_train.argtypes = [sp] + [vp] * 14 + [vp]
+        L.rola_attention_bwd_workspace_bytes.restype = sz
+        L.rola_attention_bwd_workspace_bytes.argtypes = [sp]
+        L.rola_attention_bwd.restype = ctypes.c_int
+        L.rola_attention_bwd.argtypes = [sp] + [vp] * 19 + [vp, sz, vp, vp]
         L.rola_layer_kernel_launches.restype = ctypes.c_int
         L.rola_layer_kernel_launches.argtypes = [sp]
         L.rola_layer_fwd_host.restype = ctypes.c_int
@@ -121,6 +139,12 @@ def lib() -> ctypes.CDLL:
         L.fp8_linear_workspace_bytes.argtypes = [i32, i32]
         L.fp8_linear_w8a8.restype = ctypes.c_int
         L.fp8_linear_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, sz, vp, vp]
+        L.fp8_gemm_w8a8_act.restype = ctypes.c_int
+        L.fp8_gemm_w8a8_act.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp, vp, vp]
+        L.fp8_ffn_workspace_bytes.restype = sz
+        L.fp8_ffn_workspace_bytes.argtypes = [i32, i32, i32]
+        L.fp8_ffn_w8a8.restype = ctypes.c_int
+        L.fp8_ffn_w8a8.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         _lib = L
     return _lib
 
@@ -204,8 +228,11 @@ def block_states(shape: Shape, k, v, P, *, stream=None):
 
 
 def attention_fwd(shape: Shape, q, k, v, idx, P, states, gate, *, out=None, dev_err=None,
-                  stream=None):
-    """RoLA attention output bf16 [B, N, H, d] for a given block mask."""
+                  stream=None, wait_limit_ns=None):
+    """RoLA attention output bf16 [B, N, H, d] for a given block mask.
+    ``wait_limit_ns`` bounds each pipeline wait of the kernel (default 1 s;
+    0 gives up at the first wait that is not ready, for tests of the timeout
+    path)."""
     act = (shape.B, shape.N, shape.H, shape.d)
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, act, nm)
@@ -221,11 +248,54 @@ def attention_fwd(shape: Shape, q, k, v, idx, P, states, gate, *, out=None, dev_
     if out is None:
         out = torch.empty(act, dtype=torch.bfloat16, device=q.device)
     _need(out, torch.bfloat16, act, "out")
-    _check(lib().rola_attention_fwd(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
-                                    _ptr(P), _ptr(S_blk), _ptr(z_blk), _ptr(S_glb), _ptr(z_glb),
-                                    _ptr(gate), _ptr(out), _ptr(dev_err), _stream(stream)),
-           "rola_attention_fwd")
+    args = (ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(P), _ptr(S_blk),
+            _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate), _ptr(out), _ptr(dev_err))
+    if wait_limit_ns is None:
+        _check(lib().rola_attention_fwd(*args, _stream(stream)), "rola_attention_fwd")
+    else:
+        _check(lib().rola_attention_fwd_bounded(*args, ctypes.c_uint64(int(wait_limit_ns)), _stream(stream)),
+               "rola_attention_fwd_bounded")
     return out
+
+
+def attention_fwd_train(shape: Shape, q, k, v, idx, P, states, gate, *, dev_err=None, stream=None):
+    """Forward that also returns the statistics the backward reads:
+    (out bf16 [B, N, H, d], lse float [B, H, N], den float [B, H, N])."""
+    act = (shape.B, shape.N, shape.H, shape.d)
+    S_blk, z_blk, S_glb, z_glb = states
+    out = torch.empty(act, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=q.device)
+    den = torch.empty_like(lse)
+    _check(lib().rola_attention_fwd_train(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(P),
+                                          _ptr(S_blk), _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate),
+                                          _ptr(out), _ptr(lse), _ptr(den), _ptr(dev_err), _stream(stream)),
+           "rola_attention_fwd_train")
+    return out, lse, den
+
+
+def attention_bwd(shape: Shape, q, k, v, idx, P, states, gate, out, lse, den, dout, *, dev_err=None,
+                  stream=None, workspace=None):
+    """Gradients (dq, dk, dv bf16 [B, N, H, d], dP float [H, d, r], dgate
+    float [H]) of sum(dout * out) for the forward of attention_fwd_train."""
+    act = (shape.B, shape.N, shape.H, shape.d)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _need(t, torch.bfloat16, act, nm)
+    S_blk, z_blk, S_glb, z_glb = states
+    dq, dk, dv = (torch.zeros(act, dtype=torch.bfloat16, device=q.device) for _ in range(3))
+    dP = torch.empty((shape.H, shape.d, shape.r), dtype=torch.float32, device=q.device)
+    dgate = torch.empty((shape.H,), dtype=torch.float32, device=q.device)
+    c = shape.c()
+    nbytes = lib().rola_attention_bwd_workspace_bytes(ctypes.byref(c))
+    if nbytes == 0:
+        raise RolaError("rola_attention_bwd: unsupported shape")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _ws(nbytes, q.device)
+    _check(lib().rola_attention_bwd(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(P), _ptr(S_blk),
+                                    _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate), _ptr(out), _ptr(lse),
+                                    _ptr(den), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dP), _ptr(dgate),
+                                    _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream)),
+           "rola_attention_bwd")
+    return dq, dk, dv, dP, dgate
 
 
 class Layer:
@@ -272,6 +342,39 @@ class Layer:
                                               self.ws_bytes, _ptr(self.dev_err), _stream(stream), ev,
                                               len(events)),
                    "rola_layer_fwd_timed")
+        return out
+
+
+    def run_ex(self, q, k, v, P, gate, idx, *, kb_per_head=None, reuse_mask=False, out=None,
+               stream=None, events=None):
+        """The layer with options: ``kb_per_head`` (int32 [H] on the device,
+        each in 1..k_b) keeps a different number of blocks per head;
+        ``reuse_mask`` takes ``idx`` (int32 [B, H, n_blocks, k_b]) as the mask
+        instead of selecting one (else the selected mask is written to it)."""
+        s = self.shape
+        act = (s.B, s.N, s.H, s.d)
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            _need(t, torch.bfloat16, act, nm)
+        _need(P, torch.bfloat16, (s.H, s.d, s.r), "P")
+        _need(gate, torch.float32, (s.H,), "gate")
+        _need(idx, torch.int32, (s.B, s.H, s.n_blocks, s.k_b), "idx")
+        if kb_per_head is not None:
+            _need(kb_per_head, torch.int32, (s.H,), "kb_per_head")
+        if out is None:
+            out = torch.empty(act, dtype=torch.bfloat16, device=q.device)
+        opts = LayerOpts(None if kb_per_head is None else kb_per_head.data_ptr(), 1 if reuse_mask else 0)
+        ev, n_ev = None, 0
+        if events is not None:
+            if len(events) not in (3, 5):
+                raise ValueError("events: three or five torch.cuda.Event")
+            for e in events:
+                if not e.cuda_event:
+                    e.record(stream if stream is not None else torch.cuda.current_stream())
+            ev, n_ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events]), len(events)
+        _check(lib().rola_layer_fwd_ex(ctypes.byref(self.c), ctypes.byref(opts), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(P), _ptr(gate), _ptr(out), _ptr(idx), _ptr(self.ws), self.ws_bytes,
+                                       _ptr(self.dev_err), _stream(stream), ev, n_ev),
+               "rola_layer_fwd_ex")
         return out
 
 
@@ -333,7 +436,8 @@ def fp8_quantize_weight(w, *, stream=None):
     return wq, sc
 
 
-def fp8_gemm(xq, xs, wq, ws, *, out=None, dev_err=None, stream=None):
+def fp8_gemm(xq, xs, wq, ws, *, out=None, dev_err=None, stream=None, act=ACT_NONE):
+    """y = bf16(act((x_q w_q^T) x_scale w_scale)); act ACT_NONE or ACT_GELU_TANH."""
     M, K = xq.shape
     N = wq.shape[0]
     _need(xq, torch.uint8, (M, K), "x_q")
@@ -343,8 +447,12 @@ def fp8_gemm(xq, xs, wq, ws, *, out=None, dev_err=None, stream=None):
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
     _need(out, torch.bfloat16, (M, N), "y")
-    _check(lib().fp8_gemm_w8a8(M, N, K, _ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(out),
-                               _ptr(dev_err), _stream(stream)), "fp8_gemm_w8a8")
+    if act == ACT_NONE:
+        _check(lib().fp8_gemm_w8a8(M, N, K, _ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), _ptr(out),
+                                   _ptr(dev_err), _stream(stream)), "fp8_gemm_w8a8")
+    else:
+        _check(lib().fp8_gemm_w8a8_act(M, N, K, _ptr(xq), _ptr(xs), _ptr(wq), _ptr(ws), act, _ptr(out),
+                                       _ptr(dev_err), _stream(stream)), "fp8_gemm_w8a8_act")
     return out
 
 
@@ -361,4 +469,25 @@ def fp8_linear(x, wq, ws, *, out=None, workspace=None, dev_err=None, stream=None
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _check(lib().fp8_linear_w8a8(M, N, K, _ptr(x), _ptr(wq), _ptr(ws), _ptr(out), _ptr(workspace),
                                  nbytes, _ptr(dev_err), _stream(stream)), "fp8_linear_w8a8")
+    return out
+
+
+def fp8_ffn(x, w1q, w1s, w2q, w2s, *, out=None, workspace=None, dev_err=None, stream=None):
+    """y = W2 gelu_tanh(W1 x) with both projections in W8A8 FP8: x bf16 [M, D],
+    w1q uint8 [F, D], w2q uint8 [D, F], per-output-channel float32 scales."""
+    M, D = x.shape
+    F = w1q.shape[0]
+    _need(x, torch.bfloat16, (M, D), "x")
+    _need(w1q, torch.uint8, (F, D), "w1_q")
+    _need(w1s, torch.float32, (F,), "w1_scale")
+    _need(w2q, torch.uint8, (D, F), "w2_q")
+    _need(w2s, torch.float32, (D,), "w2_scale")
+    nbytes = lib().fp8_ffn_workspace_bytes(M, D, F)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _ws(nbytes, x.device)
+    if out is None:
+        out = torch.empty((M, D), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, (M, D), "y")
+    _check(lib().fp8_ffn_w8a8(M, D, F, _ptr(x), _ptr(w1q), _ptr(w1s), _ptr(w2q), _ptr(w2s), _ptr(out),
+                              _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream)), "fp8_ffn_w8a8")
     return out

@@ -167,12 +167,17 @@ extern "C" rola_status_t rola_layer_fwd(const rola_shape_t* s, const uint16_t* q
   return rola_layer_fwd_timed(s, q, k, v, P, gate, out, idx_out, ws, ws_bytes, dev_err, stream, nullptr, 0);
 }
 
-extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint16_t* q,
-                                              const uint16_t* k, const uint16_t* v, const uint16_t* P,
-                                              const float* gate, uint16_t* out, int32_t* idx_out,
-                                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream,
-                                              void* const* events, int32_t n_events) {
+namespace {
+// The layer: selection (or a given mask), block states, attention.  kb_h:
+// optional per-head kept counts (device int32 [H]); reuse: idx_io is the mask
+// to use and no selection runs; otherwise the selected mask is copied to
+// idx_io when it is not NULL.
+rola_status_t layer_run(const rola_shape_t* s, const int32_t* kb_h, bool reuse, const uint16_t* q,
+                        const uint16_t* k, const uint16_t* v, const uint16_t* P, const float* gate,
+                        uint16_t* out, int32_t* idx_io, void* ws, size_t ws_bytes, int32_t* dev_err,
+                        void* stream, void* const* events, int32_t n_events) {
   if (events && n_events != 3 && n_events != 5) return ROLA_ERR_INVALID_ARG;
+  if (reuse && (!idx_io || !rola_host::aligned(idx_io, 4))) return idx_io ? ROLA_ERR_ALIGNMENT : ROLA_ERR_INVALID_ARG;
   // stage boundaries 0..4 (start, after the q/k/v pass, after scores and
   // top-k, after the totals, end); three events keep stages 0, 3 and 4
   auto mark = [&](int stage) -> bool {
@@ -186,7 +191,7 @@ extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint1
   const rola_internal::LayerWs L = rola_internal::layer_ws(s);
   if (!ws || ws_bytes < L.total || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
   char* base = reinterpret_cast<char*>(ws);
-  int32_t* idx = reinterpret_cast<int32_t*>(base + L.idx);
+  int32_t* idx = reuse ? idx_io : reinterpret_cast<int32_t*>(base + L.idx);
   float* S_blk = reinterpret_cast<float*>(base + L.S_blk);
   float* z_blk = reinterpret_cast<float*>(base + L.z_blk);
   float* S_glb = reinterpret_cast<float*>(base + L.S_glb);
@@ -207,30 +212,56 @@ extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint1
     st = rola::launch_prep_kernel(s, q, k, v, P, qbar, kbar, S_blk, z_blk, dev_err, cs);
     if (st != ROLA_OK) return st;
     if (!mark(1)) return ROLA_ERR_CUDA;
-    st = rola::select_from_pooled(s, qbar, kbar, sigma, idx, cs);
-    if (st != ROLA_OK) return st;
+    if (!reuse) {
+      st = rola::select_from_pooled(s, qbar, kbar, sigma, idx, cs, kb_h, dev_err);
+      if (st != ROLA_OK) return st;
+    }
     if (!mark(2)) return ROLA_ERR_CUDA;
     st = rola::launch_states_total(s, S_blk, z_blk, S_glb, z_glb, cs);
     if (st != ROLA_OK) return st;
   } else {
-    st = rola_select_blocks(s, q, k, idx, nullptr, base + L.select, L.idx - L.select, stream);
-    if (st != ROLA_OK) return st;
+    if (!reuse) {
+      st = rola::select_blocks_impl(s, kb_h, q, k, idx, nullptr, base + L.select, L.idx - L.select, dev_err,
+                                    stream);
+      if (st != ROLA_OK) return st;
+    }
     if (!mark(1) || !mark(2)) return ROLA_ERR_CUDA;
     st = rola_block_states(s, k, v, P, S_blk, z_blk, S_glb, z_glb, stream);
     if (st != ROLA_OK) return st;
   }
   if (!mark(3)) return ROLA_ERR_CUDA;
-  st = rola_attention_fwd(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
-                          stream);
+  st = rola::attention_launch(s, kb_h, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
+                              rola::kWaitLimitNs, stream);
   if (st != ROLA_OK) return st;
   if (!mark(4)) return ROLA_ERR_CUDA;
-  if (idx_out) {
+  if (idx_io && !reuse) {
     const size_t bytes = (size_t)s->B * s->H * rola_num_blocks(s) * s->k_b * sizeof(int32_t);
-    if (cudaMemcpyAsync(idx_out, idx, bytes, cudaMemcpyDeviceToDevice,
+    if (cudaMemcpyAsync(idx_io, idx, bytes, cudaMemcpyDeviceToDevice,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
       return ROLA_ERR_CUDA;
   }
   return ROLA_OK;
+}
+}  // namespace
+
+extern "C" rola_status_t rola_layer_fwd_timed(const rola_shape_t* s, const uint16_t* q,
+                                              const uint16_t* k, const uint16_t* v, const uint16_t* P,
+                                              const float* gate, uint16_t* out, int32_t* idx_out,
+                                              void* ws, size_t ws_bytes, int32_t* dev_err, void* stream,
+                                              void* const* events, int32_t n_events) {
+  return layer_run(s, nullptr, false, q, k, v, P, gate, out, idx_out, ws, ws_bytes, dev_err, stream, events,
+                   n_events);
+}
+
+extern "C" rola_status_t rola_layer_fwd_ex(const rola_shape_t* s, const rola_layer_opts_t* opts,
+                                           const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                           const uint16_t* P, const float* gate, uint16_t* out,
+                                           int32_t* idx_io, void* ws, size_t ws_bytes, int32_t* dev_err,
+                                           void* stream, void* const* events, int32_t n_events) {
+  const int32_t* kb_h = opts ? opts->kb_per_head : nullptr;
+  if (kb_h && !rola_host::aligned(kb_h, 4)) return ROLA_ERR_ALIGNMENT;
+  return layer_run(s, kb_h, opts && opts->reuse_mask, q, k, v, P, gate, out, idx_io, ws, ws_bytes, dev_err,
+                   stream, events, n_events);
 }
 
 namespace {

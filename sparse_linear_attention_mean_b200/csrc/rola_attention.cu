@@ -93,12 +93,14 @@ struct AttnParams {
   const float* gate;
   uint16_t* out;
   int32_t* dev_err;
+  uint64_t wait_ns;  // bound of each pipeline wait (0: give up at the first wait that finds its stage not ready)
+  const int32_t* kb_h;  // per-head kept counts (NULL: kb for every head); idx rows keep stride kb
   RopeTable rope;
 };
 
 // All lanes wait; the warp agrees on the outcome (and reconverges).
-ROLA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+ROLA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -124,8 +126,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = (size_t)b * p.H + h;
 
-  // A CTA that already timed out in this launch makes the rest skip their work.
-  if (p.dev_err && (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)) return;
+  // A CTA that already timed out in this launch makes the rest skip their
+  // work; the barrier gives every thread of the CTA the same answer.
+  if (__syncthreads_or(tid == 0 && p.dev_err &&
+                       (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)))
+    return;
+  const uint64_t lim = p.wait_ns;  // bound of each pipeline wait
 
   // ------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -153,9 +159,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(&M.tmem_base, L::TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = tid; i < QB * p.kb; i += kAttnThreads) {
-    const int qb = i / p.kb, a = tile * QB + qb;
-    M.raw[qb][i % p.kb] = a < p.nb ? p.idx[(bh * p.nb + a) * p.kb + i % p.kb] : -1;
+  // this head's kept count (a count outside [1, kb] is clamped and reported)
+  const int kb_want = p.kb_h ? p.kb_h[h] : p.kb;
+  const int kbh = min(max(kb_want, 1), p.kb);
+  for (int i = tid; i < QB * kbh; i += kAttnThreads) {
+    const int qb = i / kbh, a = tile * QB + qb;
+    M.raw[qb][i % kbh] = a < p.nb ? p.idx[(bh * p.nb + a) * p.kb + i % kbh] : -1;
   }
   // P_h^T as a K-major (N = r rows, K = d) operand with 128-byte swizzle.
   {
@@ -182,9 +191,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       pos[qb] = 0;
       prev[qb] = -1;
       M.cnt[qb] = 0;
-      len[qb] = (tile * QB + qb) < p.nb ? p.kb : 0;
+      len[qb] = (tile * QB + qb) < p.nb ? kbh : 0;
     }
-    int nk = 0, err = 0;
+    int nk = 0, err = kbh != kb_want;
     while (true) {
       int best = 0x7fffffff;
       for (int qb = 0; qb < QB; ++qb) {
@@ -233,7 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int j = 0;
       for (; j < nk; ++j) {
         const int st = j % L::NS;
-        if (j >= L::NS && !mbar_wait(&M.kv_empty[st], ((j / L::NS) - 1) & 1, abort)) break;
+        if (j >= L::NS && !mbar_wait(&M.kv_empty[st], ((j / L::NS) - 1) & 1, abort, lim)) break;
         const int u = M.ulist[j];
         mbar_expect_tx(&M.k_full[st], L::KV_BYTES);
         for (int ka = 0; ka < L::KA; ++ka)
@@ -269,9 +278,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
       auto issue_pv = [&](int i) -> bool {
         const int sb = i & 1, st = i % L::NS;
-        if (!mbar_wait(&M.p_full[sb], (i >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&M.o_ready, i & 1, abort)) return false;
-        if (!mbar_wait(&M.v_full[st], (i / L::NS) & 1, abort)) return false;
+        if (!mbar_wait(&M.p_full[sb], (i >> 1) & 1, abort, lim)) return false;
+        if (!mbar_wait(&M.o_ready, i & 1, abort, lim)) return false;
+        if (!mbar_wait(&M.v_full[st], (i / L::NS) & 1, abort, lim)) return false;
         tc_fence_after();
         const uint32_t vbase = sV + st * L::KV_BYTES;
 #pragma unroll
@@ -285,7 +294,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         return true;
       };
 
-      bool ok = mbar_wait(&M.bar_q, 0, abort);
+      bool ok = mbar_wait(&M.bar_q, 0, abort, lim);
       if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -296,10 +305,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       for (int j = 0; ok && j < nk; ++j) {
         const int st = j % L::NS, sb = j & 1;
-        ok = mbar_wait(&M.k_full[st], (j / L::NS) & 1, abort);
+        ok = mbar_wait(&M.k_full[st], (j / L::NS) & 1, abort, lim);
         // The S buffer about to be overwritten still holds P_{j-2}; let that
         // P.V finish first.
-        if (ok && j >= 2) ok = mbar_wait(&M.pv_done, (j - 2) & 1, abort);
+        if (ok && j >= 2) ok = mbar_wait(&M.pv_done, (j - 2) & 1, abort, lim);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kbase = sK + st * L::KV_BYTES;
@@ -311,8 +320,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j >= 1) ok = issue_pv(j - 1);
       }
       if (ok && nk > 0) ok = issue_pv(nk - 1);
-      if (ok) ok = mbar_wait(&M.lin_ready, 0, abort);
-      if (ok && nk > 0) ok = mbar_wait(&M.pv_done, (nk - 1) & 1, abort);
+      if (ok) ok = mbar_wait(&M.lin_ready, 0, abort, lim);
+      if (ok && nk > 0) ok = mbar_wait(&M.pv_done, (nk - 1) & 1, abort, lim);
       if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       const int sb = j & 1;
-      if (!warp_wait(&M.s_full[sb], (j >> 1) & 1, abort)) {
+      if (!warp_wait(&M.s_full[sb], (j >> 1) & 1, abort, lim)) {
         ok = false;
         break;
       }
@@ -399,7 +408,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int n = tile * L::BM + row;
     mbar_arrive(&M.o_ready);  // iteration 0: nothing to rescale
     float psi[R];
-    bool ok = warp_wait(&M.qt_full, 0, abort);
+    bool ok = warp_wait(&M.qt_full, 0, abort, lim);
     if (ok) {
       tc_fence_after();
       uint32_t qt[32];
@@ -436,10 +445,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int j = 1; ok && j < nk; ++j) {
       const int sb = j & 1;
-      ok = warp_wait(&M.scale_ready[sb], (j >> 1) & 1, abort);
+      ok = warp_wait(&M.scale_ready[sb], (j >> 1) & 1, abort, lim);
       if (!ok) break;
       const float alpha = M.scale[sb][row];
-      ok = warp_wait(&M.pv_done, (j - 1) & 1, abort);
+      ok = warp_wait(&M.pv_done, (j - 1) & 1, abort, lim);
       if (!ok) break;
       tc_fence_after();
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -457,9 +466,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(&M.o_ready);
     }
-    if (ok) ok = warp_wait(&M.stats_ready, 0, abort);
-    if (ok && nk > 0) ok = warp_wait(&M.pv_done, (nk - 1) & 1, abort);
-    if (ok) ok = warp_wait(&M.l_done, 0, abort);
+    if (ok) ok = warp_wait(&M.stats_ready, 0, abort, lim);
+    if (ok && nk > 0) ok = warp_wait(&M.pv_done, (nk - 1) & 1, abort, lim);
+    if (ok) ok = warp_wait(&M.l_done, 0, abort, lim);
     if (ok) {
       tc_fence_after();
       const float lsum = M.rowl[row];
@@ -590,19 +599,19 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
                                  const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                  const float* S_blk, const float* z_blk, const float* S_glb,
                                  const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
+                                 const int32_t* kb_h, uint64_t wait_ns, float* lse, float* den,
                                  cudaStream_t cs);
 
 }  // namespace rola
 
 using namespace rola;
 
-extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_t* q,
-                                            const uint16_t* k, const uint16_t* v,
-                                            const int32_t* idx, const uint16_t* P,
-                                            const float* S_blk, const float* z_blk,
-                                            const float* S_glb, const float* z_glb,
-                                            const float* gate, uint16_t* out, int32_t* dev_err,
-                                            void* stream) {
+rola_status_t rola::attention_launch(const rola_shape_t* s, const int32_t* kb_h, const uint16_t* q,
+                                     const uint16_t* k, const uint16_t* v, const int32_t* idx,
+                                     const uint16_t* P, const float* S_blk, const float* z_blk,
+                                     const float* S_glb, const float* z_glb, const float* gate,
+                                     uint16_t* out, int32_t* dev_err, uint64_t wait_limit_ns,
+                                     void* stream) {
   rola_status_t st = rola_internal::check_shape(s);
   if (st != ROLA_OK) return st;
   if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out)
@@ -629,12 +638,15 @@ extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_
   prm.gate = gate;
   prm.out = out;
   prm.dev_err = dev_err;
+  prm.wait_ns = wait_limit_ns;
+  prm.kb_h = kb_h;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   // the two-tile kernel reads the states with 32-byte loads and P_h with 16-byte loads
   if (pair_kernel_supports(s) && rola_host::aligned(S_blk, 32) && rola_host::aligned(S_glb, 32) &&
       rola_host::aligned(P, 16))
-    return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, cs);
+    return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, kb_h,
+                              wait_limit_ns, nullptr, nullptr, cs);
   if (s->d == 128 && s->block == 128 && s->r == 32) return launch_attn<128, 128, 32>(s, q, k, v, prm, cs);
   if (s->d == 128 && s->block == 128 && s->r == 16) return launch_attn<128, 128, 16>(s, q, k, v, prm, cs);
   if (s->d == 64 && s->block == 64 && s->r == 16) return launch_attn<64, 64, 16>(s, q, k, v, prm, cs);
@@ -642,4 +654,48 @@ extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_
   if (s->d == 64 && s->block == 128 && s->r == 16) return launch_attn<64, 128, 16>(s, q, k, v, prm, cs);
   if (s->d == 64 && s->block == 128 && s->r == 32) return launch_attn<64, 128, 32>(s, q, k, v, prm, cs);
   return ROLA_ERR_UNSUPPORTED;
+}
+
+extern "C" rola_status_t rola_attention_fwd_bounded(const rola_shape_t* s, const uint16_t* q,
+                                                    const uint16_t* k, const uint16_t* v,
+                                                    const int32_t* idx, const uint16_t* P,
+                                                    const float* S_blk, const float* z_blk,
+                                                    const float* S_glb, const float* z_glb,
+                                                    const float* gate, uint16_t* out,
+                                                    int32_t* dev_err, uint64_t wait_limit_ns,
+                                                    void* stream) {
+  return attention_launch(s, nullptr, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
+                          wait_limit_ns, stream);
+}
+
+extern "C" rola_status_t rola_attention_fwd(const rola_shape_t* s, const uint16_t* q,
+                                            const uint16_t* k, const uint16_t* v,
+                                            const int32_t* idx, const uint16_t* P,
+                                            const float* S_blk, const float* z_blk,
+                                            const float* S_glb, const float* z_glb,
+                                            const float* gate, uint16_t* out, int32_t* dev_err,
+                                            void* stream) {
+  return rola_attention_fwd_bounded(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err,
+                                    kWaitLimitNs, stream);
+}
+
+extern "C" rola_status_t rola_attention_fwd_train(const rola_shape_t* s, const uint16_t* q,
+                                                  const uint16_t* k, const uint16_t* v,
+                                                  const int32_t* idx, const uint16_t* P,
+                                                  const float* S_blk, const float* z_blk,
+                                                  const float* S_glb, const float* z_glb,
+                                                  const float* gate, uint16_t* out, float* lse,
+                                                  float* den, int32_t* dev_err, void* stream) {
+  rola_status_t st = rola_internal::check_shape(s);
+  if (st != ROLA_OK) return st;
+  if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out || !lse || !den)
+    return ROLA_ERR_INVALID_ARG;
+  if (!pair_kernel_supports(s)) return ROLA_ERR_UNSUPPORTED;
+  if (!rola_host::aligned(q, 16) || !rola_host::aligned(k, 16) || !rola_host::aligned(v, 16) ||
+      !rola_host::aligned(out, 16) || !rola_host::aligned(S_blk, 32) || !rola_host::aligned(S_glb, 32) ||
+      !rola_host::aligned(idx, 4) || !rola_host::aligned(P, 16) || !rola_host::aligned(lse, 4) ||
+      !rola_host::aligned(den, 4))
+    return ROLA_ERR_ALIGNMENT;
+  return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, nullptr,
+                            kWaitLimitNs, lse, den, reinterpret_cast<cudaStream_t>(stream));
 }

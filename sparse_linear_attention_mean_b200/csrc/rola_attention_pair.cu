@@ -54,11 +54,6 @@ constexpr int NR = 3;                   // K/V ring slots (each one K or one V t
 constexpr int D = 128, BM = 128, BN = 128;
 constexpr uint32_t TILE = BM * D * 2;   // 32 KB: one Q, K or V tile
 constexpr float kRescaleThreshold = 8.f;  // log2 units
-// Moving every kEmuEvery-th exp2 pair onto the FMA pipe (exp2_poly2) was
-// measured slower on B200 for this kernel (the softmax is not bound by the
-// special-function unit), so it is off.
-constexpr bool kEmuExp2 = false;
-constexpr int kEmuEvery = 4;
 
 template <int R>
 struct Layout {
@@ -80,14 +75,24 @@ struct Layout {
 constexpr int NL = 3;        // unit lists in flight: the producer builds one unit ahead
 constexpr int kMaxBlocks = 1024;  // n_blocks limit (the list merge keeps one bit per block)
 
+constexpr uint16_t kNoBlock = 0xffff;
+
+// One unit's work lists.  The union (ascending, with a per-slot mask) drives
+// the state gather.  The steps drive the tensor-core pipeline: in step j slot
+// s works on key block sblk[s][j] (kNoBlock: slot idle).  A block both slots
+// keep is one shared step (its K and V tiles serve both); the blocks only one
+// slot keeps are paired across the slots, each step then loading two K/V
+// pairs, so that both slots have a tile in almost every step.
 struct UnitList {
   int b, h, a[2];
   int active[2];
-  int nu;
+  int nu;  // union entries
+  int ns;  // steps
   int cnt[2];
   int lin_empty[2];
   uint16_t ulist[kMaxUnion];
   uint8_t umask[kMaxUnion];
+  uint16_t sblk[2][kMaxKept];
 };
 
 constexpr int kTabCap = 1024;  // cos/sin entries of the rotary table in shared memory
@@ -122,6 +127,10 @@ struct Params {
   uint16_t* out;
   int out_32b;  // out is 32-byte aligned: the epilogue stores 32 bytes at a time
   int32_t* dev_err;
+  uint64_t wait_ns;  // bound of each pipeline wait (0: give up at the first wait that finds its stage not ready)
+  const int32_t* kb_h;  // per-head kept counts (NULL: kb for every head); idx rows keep stride kb
+  float* lse;  // optional [B, H, N]: natural log-sum-exp of the scaled kept scores per row
+  float* den;  // optional [B, H, N]: linear denominator psi_q . z_U (NaN when the complement is empty)
   RopeTable rope;
   // rotary table: entry of pair pr at position pos = tab_base[pr] + pos * tab_stride[pr];
   // pair pr fills entries [tab_first[pr], tab_first[pr + 1]) of the fill order
@@ -132,8 +141,8 @@ struct Params {
 ROLA_DEV uint32_t s_col(int s) { return (uint32_t)s * 128u; }
 ROLA_DEV uint32_t o_col(int s) { return 256u + (uint32_t)s * 128u; }
 
-ROLA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+ROLA_DEV bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 ROLA_DEV uint64_t desc_k_sw128(uint32_t base, int rows, int kk) {
@@ -176,7 +185,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   Misc& M = *reinterpret_cast<Misc*>(smem + Ly::misc_off);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  if (p.dev_err && (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)) return;
+  // A CTA that already timed out in this launch makes the rest skip their
+  // work; the barrier gives every thread of the CTA the same answer.
+  if (__syncthreads_or(tid == 0 && p.dev_err &&
+                       (*reinterpret_cast<volatile int32_t*>(p.dev_err) & ROLA_DEVERR_TIMEOUT)))
+    return;
+  const uint64_t lim = p.wait_ns;  // bound of each pipeline wait
 
   if (tid == 0) {
     for (int i = 0; i < NL; ++i) {
@@ -239,14 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int u = 0; ok && u < my_units; ++u) {
       const int buf = u % NL;
-      if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
+      if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort, lim))) break;
       const UnitList& U = M.L[buf];
       if (U.active[s]) {
         float m = 0.f, l = 0.f;
         bool first = true;
-        for (int j = 0; j < U.nu; ++j) {
-          if (!((U.umask[j] >> s) & 1)) continue;
-          if (!(ok = warp_wait(&M.s_full[s], nsc & 1, abort))) break;
+        for (int j = 0; j < U.ns; ++j) {
+          const int blk = U.sblk[s][j];
+          if (blk == kNoBlock) continue;
+          if (!(ok = warp_wait(&M.s_full[s], nsc & 1, abort, lim))) break;
           ++nsc;
           tc_fence_after();
           uint32_t x[128];
@@ -255,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32_at<64>(sc + 64, x);
           tmem_ld32_at<96>(sc + 96, x);
           tmem_wait_ld();
-          const int blk = U.ulist[j];
           if (blk == p.nb - 1) {
             // padded keys of the last block take no part in the softmax
             const int valid = p.N - blk * BN;
@@ -288,14 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint64_t acc2 = f32x2(0.f, 0.f);
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
-            float y0, y1, p0, p1;
+            float y0, y1;
             f32x2_split(ffma2(f32x2(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2, nm2), y0, y1);
-            if (kEmuExp2 && (c >> 1) % kEmuEvery == kEmuEvery - 1) {
-              exp2_poly2(y0, y1, p0, p1);  // FMA pipe
-            } else {
-              p0 = fast_exp2(y0);          // special-function unit
-              p1 = fast_exp2(y1);
-            }
+            const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
             acc2 = fadd2(acc2, f32x2(p0, p1));
             x[c >> 1] = pack_bf16(p0, p1);
           }
@@ -331,14 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // that MMA; q P_h sits in columns [0, r).
         // This code runs once per unit, cold in the instruction cache, so it
         // is written as short rolled loops over 8-column chunks.
-        if (!(ok = warp_wait(&M.qt_full[s], uc & 1, abort))) break;
+        if (!(ok = warp_wait(&M.qt_full[s], uc & 1, abort, lim))) break;
         tc_fence_after();
         const int n = U.a[s] * BM + row;
         const int nn = n < p.N ? n : p.N - 1;
         const int hw = p.Hg * p.W;
         const int pt_ = nn / hw, rem = nn - pt_ * hw;
         const int py = rem / p.W, px = rem - py * p.W;
-        if (!(ok = warp_wait(&M.zu_ready[s], uc & 1, abort))) break;
+        if (!(ok = warp_wait(&M.zu_ready[s], uc & 1, abort, lim))) break;
         // pass 1: den = psi_q . z_U
         float den = 0.f;
 #pragma unroll 1
@@ -352,6 +361,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool have_o = U.cnt[s] > 0;
         const float lsum = have_o ? l : 1.f;
         const float scale = U.lin_empty[s] ? 0.f : p.gate[U.h] * lsum / den;
+        if (p.lse && n < p.N) {
+          // statistics a backward pass reads: sum_j exp(s_j / sqrt(d)) = 2^m l
+          const size_t ro = ((size_t)U.b * p.H + U.h) * p.N + n;
+          p.lse[ro] = have_o ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          p.den[ro] = U.lin_empty[s] ? __int_as_float(0x7fc00000) : den;
+        }
         // pass 2: rho'_q = R(t, y, x) psi_q * scale as bf16 hi + lo
 #pragma unroll 1
         for (int c8 = 0; c8 < R / 8; ++c8) {
@@ -375,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&M.lin_ready[s]);
         // ---- epilogue: out = O / l
-        if (!(ok = warp_wait(&M.l_done[s], uc & 1, abort))) break;
+        if (!(ok = warp_wait(&M.l_done[s], uc & 1, abort, lim))) break;
         tc_fence_after();
         const float inv_l = 1.f / lsum;
         const bool write = n < p.N;
@@ -424,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = 0; ok && u < my_units; ++u) {
         const int buf = u % NL;
-        if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
+        if (!(ok = warp_wait(&M.list_full[buf], (u / NL) & 1, abort, lim))) break;
         const UnitList& U = M.L[buf];
         const int b = U.b, h = U.h;
         const size_t bh = (size_t)b * p.H + h;
@@ -443,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (and its q P_h MMAs read P_h^T) -- wait for them
 #pragma unroll
         for (int s = 0; s < 2; ++s)
-          if (ok && uc[s] >= 1) ok = warp_wait(&M.l_done[s], (uc[s] - 1) & 1, abort);
+          if (ok && uc[s] >= 1) ok = warp_wait(&M.l_done[s], (uc[s] - 1) & 1, abort, lim);
         if (!ok) break;
         // P_h^T (K-major, N = r rows, K = d, 128-byte swizzle), rewritten only
         // when the head changes; P_h is read 8 values (16 bytes) at a time
@@ -509,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < PER; ++i) v[i] = a[t + 64 * i];
           // every thread has read its part before anyone overwrites the region
           mbar_arrive(&M.cvt[s]);
-          if (!(ok = warp_wait(&M.cvt[s], uc[s] & 1, abort))) continue;
+          if (!(ok = warp_wait(&M.cvt[s], uc[s] & 1, abort, lim))) continue;
           uint8_t* su_hi = reinterpret_cast<uint8_t*>(a);
           uint8_t* su_lo = su_hi + Ly::SU_BYTES;
 #pragma unroll
@@ -546,10 +561,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Unit list of unit u into buffer u % NL, by the whole warp: both kept
       // lists are validated (in range, above the previous entry of the row;
       // a bad entry is skipped and reported), marked in one bitmap per slot
-      // and read back as one ascending union with a per-slot mask.
+      // and read back as one ascending union with a per-slot mask, and as the
+      // steps: the n_sh blocks both slots keep and the n_sp = min(n_0, n_1)
+      // pairs of slot-only blocks alternate (shared, pair, shared, pair, ...,
+      // then the rest of the longer kind), and the slot-only blocks left over
+      // when n_0 != n_1 (a skipped bad entry, or an idle second slot) follow
+      // as single-slot steps.
       auto build_list = [&](int u) -> bool {
         const int buf = u % NL;
-        if (u >= NL && !warp_wait(&M.list_empty[buf], ((u / NL) - 1) & 1, abort)) return false;
+        if (u >= NL && !warp_wait(&M.list_empty[buf], ((u / NL) - 1) & 1, abort, lim)) return false;
         UnitList& U = M.L[buf];
         int b, h, pair;
         decode_unit(p, (int)blockIdx.x + u * (int)gridDim.x, b, h, pair);
@@ -559,8 +579,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         M.kept_bits[1][lane] = 0u;
         __syncwarp();
         int err = 0;
-        for (int i = lane; i < 2 * p.kb; i += 32) {
-          const int sl = i >= p.kb ? 1 : 0, e = i - sl * p.kb, a = sl ? a1 : a0;
+        int kbh = p.kb;  // this head's kept count (a count outside [1, kb] is clamped and reported)
+        if (p.kb_h) {
+          const int want = p.kb_h[h];
+          kbh = min(max(want, 1), p.kb);
+          err = kbh != want;
+        }
+        for (int i = lane; i < 2 * kbh; i += 32) {
+          const int sl = i >= kbh ? 1 : 0, e = i - sl * kbh, a = sl ? a1 : a0;
           if (a >= p.nb) continue;
           const int32_t* row = p.idx + (bh * p.nb + a) * p.kb;
           const int v = row[e];
@@ -571,26 +597,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         const uint32_t m0 = M.kept_bits[0][lane], m1 = M.kept_bits[1][lane], mu = m0 | m1;
-        int pre = __popc(mu);  // inclusive prefix over lanes: lane w holds blocks [32 w, 32 w + 32)
+        const uint32_t sh = m0 & m1, x0 = m0 & ~m1, x1 = m1 & ~m0;
+        // inclusive prefix counts over lanes (lane w holds blocks [32 w, 32 w + 32)),
+        // two 16-bit counts per word: union | shared << 16, slot-0-only | slot-1-only << 16
+        int pa = __popc(mu) | (__popc(sh) << 16), pb = __popc(x0) | (__popc(x1) << 16);
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-          const int t = __shfl_up_sync(0xffffffffu, pre, off);
-          if (lane >= off) pre += t;
+          const int ta = __shfl_up_sync(0xffffffffu, pa, off), tb = __shfl_up_sync(0xffffffffu, pb, off);
+          if (lane >= off) {
+            pa += ta;
+            pb += tb;
+          }
         }
-        int pos = pre - __popc(mu);
+        const int ta = __shfl_sync(0xffffffffu, pa, 31), tb = __shfl_sync(0xffffffffu, pb, 31);
+        const int nu = ta & 0xffff, nsh = ta >> 16, n0 = tb & 0xffff, n1 = tb >> 16;
+        const int nsp = min(n0, n1), mlt = min(nsh, nsp);
+        int pos = (pa & 0xffff) - __popc(mu);
         for (uint32_t rem = mu; rem; rem &= rem - 1) {
           const int bit = __ffs(rem) - 1;
           U.ulist[pos] = (uint16_t)(lane * 32 + bit);
           U.umask[pos] = (uint8_t)(((m0 >> bit) & 1u) | (((m1 >> bit) & 1u) << 1));
           ++pos;
         }
-        int c0 = __popc(m0), c1 = __popc(m1);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          c0 += __shfl_xor_sync(0xffffffffu, c0, off);
-          c1 += __shfl_xor_sync(0xffffffffu, c1, off);
+        int i = (pa >> 16) - __popc(sh);  // shared block i -> step 2 i, or 2 mlt + (i - mlt)
+        for (uint32_t rem = sh; rem; rem &= rem - 1, ++i) {
+          const int st = i < mlt ? 2 * i : 2 * mlt + (i - mlt);
+          U.sblk[0][st] = U.sblk[1][st] = (uint16_t)(lane * 32 + __ffs(rem) - 1);
         }
-        const int nu = __shfl_sync(0xffffffffu, pre, 31);
+        // slot-only block k of slot sl: pair k -> step 2 k + 1, or 2 mlt + (k - mlt);
+        // leftovers after the pairs -> single-slot steps after nsh + nsp
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          int k = sl ? (pb >> 16) - __popc(x1) : (pb & 0xffff) - __popc(x0);
+          for (uint32_t rem = sl ? x1 : x0; rem; rem &= rem - 1, ++k) {
+            const uint16_t blk = (uint16_t)(lane * 32 + __ffs(rem) - 1);
+            if (k < nsp) {
+              U.sblk[sl][k < mlt ? 2 * k + 1 : 2 * mlt + (k - mlt)] = blk;
+            } else {
+              const int st = nsh + nsp + (sl ? n0 - nsp : 0) + (k - nsp);
+              U.sblk[sl][st] = blk;
+              U.sblk[sl ^ 1][st] = kNoBlock;
+            }
+          }
+        }
+        const int c0 = nsh + n0, c1 = nsh + n1;
         if (__any_sync(0xffffffffu, err) && lane == 0) M.err = 1;
         if (lane == 0) {
           U.b = b;
@@ -600,6 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           U.active[0] = a0 < p.nb;
           U.active[1] = a1 < p.nb;
           U.nu = nu;
+          U.ns = nsh + max(n0, n1);
           U.cnt[0] = c0;
           U.cnt[1] = c1;
           U.lin_empty[0] = c0 >= p.nb;
@@ -613,31 +664,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (my_units > 0) ok = build_list(0);
       for (int u = 0; ok && u < my_units; ++u) {
         const UnitList& U = M.L[u % NL];
-        const int nu = U.nu, b = U.b, h = U.h;
-        // K and V of every union entry, gathered by block index
-        auto load_kv = [&](int j) -> bool {
-          const int blk = U.ulist[j];
-          for (int kv = 0; kv < 2; ++kv) {
-            const int slot = g % NR;
-            if (g >= (uint32_t)NR && !mbar_wait(&M.ring_empty[slot], ((g / NR) - 1) & 1, abort)) return false;
-            mbar_expect_tx(&M.ring_full[slot], TILE);
-            const CUtensorMap* mp = kv ? &tmV : &tmK;
-            for (int ka = 0; ka < 2; ++ka)
-              tma_load_4d(smem + Ly::ring_off + slot * TILE + ka * (BN * 128), mp, &M.ring_full[slot],
-                          ka * 64, h, blk * BN, b);
-            ring_par[slot] = (g / NR) & 1;
-            ++g;
-          }
+        const int ns = U.ns, b = U.b, h = U.h;
+        // one K or V tile of a key block into the next ring slot, by block index
+        auto load_tile = [&](const CUtensorMap* mp, int blk) -> bool {
+          const int slot = g % NR;
+          if (g >= (uint32_t)NR && !mbar_wait(&M.ring_empty[slot], ((g / NR) - 1) & 1, abort, lim)) return false;
+          mbar_expect_tx(&M.ring_full[slot], TILE);
+          for (int ka = 0; ka < 2; ++ka)
+            tma_load_4d(smem + Ly::ring_off + slot * TILE + ka * (BN * 128), mp, &M.ring_full[slot], ka * 64,
+                        h, blk * BN, b);
+          ring_par[slot] = (g / NR) & 1;
+          ++g;
           return true;
         };
-        // the first entry, then the Q tiles (after the previous unit's last
-        // S MMA has read them), so that the first copy overlaps the previous
-        // unit's tail
+        // the tiles of step j in the order the MMAs first use them: K then V of
+        // a shared or single-slot step; K_0, K_1, V_0, V_1 of a paired step.
+        // part 0 is the first two tiles, part 1 the rest (a pair's V tiles).
+        auto load_step = [&](int j, int part) -> bool {
+          const int b0 = U.sblk[0][j], b1 = U.sblk[1][j];
+          if (b0 != kNoBlock && b1 != kNoBlock && b0 != b1)
+            return part == 0 ? load_tile(&tmK, b0) && load_tile(&tmK, b1)
+                             : load_tile(&tmV, b0) && load_tile(&tmV, b1);
+          const int blk = b0 != kNoBlock ? b0 : b1;
+          return part == 0 ? load_tile(&tmK, blk) && load_tile(&tmV, blk) : true;
+        };
+        // the first two tiles of the first step, then the Q tiles (after the
+        // previous unit's last S MMA has read them), so that the first copies
+        // overlap the previous unit's tail, then the rest of the first step.
+        // The ring holds three tiles: a pair's fourth tile goes into the slot
+        // its first tile (K_0) frees, which needs the unit's first S MMA and
+        // so its Q tile -- Q goes out before it.
         if (lane == 0) {
-          if (nu > 0) ok = load_kv(0);
+          if (ns > 0) ok = load_step(0, 0);
           for (int sl = 0; sl < 2 && ok; ++sl) {
             if (!U.active[sl]) continue;
-            if (uc[sl] >= 1 && !(ok = mbar_wait(&M.q_empty[sl], (uc[sl] - 1) & 1, abort))) break;
+            if (uc[sl] >= 1 && !(ok = mbar_wait(&M.q_empty[sl], (uc[sl] - 1) & 1, abort, lim))) break;
             mbar_expect_tx(&M.q_full[sl], TILE);
             for (int ka = 0; ka < 2; ++ka)
               tma_load_4d(smem + Ly::q_off + sl * TILE + ka * (BM * 128), &tmQ, &M.q_full[sl], ka * 64, h,
@@ -645,12 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             q_par[sl] = uc[sl] & 1;
             ++uc[sl];
           }
+          if (ok && ns > 0) ok = load_step(0, 1);
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         // the next unit's list while this unit's copies are in flight
         if (ok && u + 1 < my_units) ok = build_list(u + 1);
         if (lane == 0)
-          for (int j = 1; ok && j < nu; ++j) ok = load_kv(j);
+          for (int j = 1; ok && j < ns; ++j) ok = load_step(j, 0) && load_step(j, 1);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         __syncwarp();
       }
@@ -680,26 +742,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dr_base = desc_k_sw128(sR, BN, 0);
       const uint64_t dv_base = smem_desc(sR, BN * 128, 1024, kSwizzle128B);
       uint32_t g = 0, np[2] = {0, 0}, uc[2] = {0, 0};
-      int users[NR];
-      for (int i = 0; i < NR; ++i) users[i] = 0;
+
       bool ok = true;
       for (int u = 0; ok && u < my_units; ++u) {
         const int buf = u % NL;
-        if (!(ok = mbar_wait(&M.list_full[buf], (u / NL) & 1, abort))) break;
+        if (!(ok = mbar_wait(&M.list_full[buf], (u / NL) & 1, abort, lim))) break;
         const UnitList& U = M.L[buf];
 #pragma unroll
         for (int s = 0; s < 2; ++s)
-          if (ok && U.active[s]) ok = mbar_wait(&M.q_full[s], uc[s] & 1, abort);
+          if (ok && U.active[s]) ok = mbar_wait(&M.q_full[s], uc[s] & 1, abort, lim);
         if (!ok) break;
         int pend_v[2] = {-1, -1};  // ring index of the V tile a slot's next P.V uses
+        // A ring tile is released by the last MMA that reads it.  Within a
+        // step slot 0's MMAs go out before slot 1's (S here, P.V in the next
+        // step or at the tile end), so a tile both slots read is released by
+        // slot 1's MMA, and a tile one slot reads by that slot's.
+        bool rel_v[2] = {false, false};
         bool first_pv[2] = {true, true};
         auto issue_pv = [&](int s) -> bool {
-          if (!mbar_wait(&M.p_full[s], np[s] & 1, abort)) return false;
+          if (!mbar_wait(&M.p_full[s], np[s] & 1, abort, lim)) return false;
           // the previous unit's epilogue must have read O first
-          if (first_pv[s] && uc[s] >= 1 && !mbar_wait(&M.o_free[s], (uc[s] - 1) & 1, abort)) return false;
+          if (first_pv[s] && uc[s] >= 1 && !mbar_wait(&M.o_free[s], (uc[s] - 1) & 1, abort, lim)) return false;
           ++np[s];
           const uint32_t gv = (uint32_t)pend_v[s];
-          if (!mbar_wait(&M.ring_full[gv % NR], (gv / NR) & 1, abort)) return false;
+          if (!mbar_wait(&M.ring_full[gv % NR], (gv / NR) & 1, abort, lim)) return false;
           tc_fence_after();
           const uint64_t dv = dv_base + (uint64_t)(gv % NR) * (TILE >> 4);
           const uint32_t acc0 = first_pv[s] ? 0u : 1u;
@@ -708,41 +774,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tm + o_col(s), tm + s_col(s) + Ly::P_OFF + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4),
                    idesc_pv, kk == 0 ? acc0 : 1u);
           first_pv[s] = false;
-          if (--users[gv % NR] == 0) mma_commit(&M.ring_empty[gv % NR]);
+          if (rel_v[s]) mma_commit(&M.ring_empty[gv % NR]);
           pend_v[s] = -1;
           return true;
         };
-        for (int j = 0; ok && j < U.nu; ++j) {
-          const uint32_t gk = g, gv = g + 1;
-          g += 2;
+        for (int j = 0; ok && j < U.ns; ++j) {
+          // the step's tiles in the producer's order: K, V (one block, used by
+          // every slot working in the step) or K_0, K_1, V_0, V_1 (a pair)
+          const int blk[2] = {U.sblk[0][j], U.sblk[1][j]};
+          const bool paired = blk[0] != kNoBlock && blk[1] != kNoBlock && blk[0] != blk[1];
+          // the one reader (paired step or idle slot) or slot 1 releases
+          const bool last[2] = {paired || blk[1] == kNoBlock, true};
+          uint32_t gk[2], gv[2];
+          if (paired) {
+            gk[0] = g;
+            gk[1] = g + 1;
+            gv[0] = g + 2;
+            gv[1] = g + 3;
+            g += 4;
+          } else {
+            gk[0] = gk[1] = g;
+            gv[0] = gv[1] = g + 1;
+            g += 2;
+          }
           // slot 0's pending P.V needs no new tile: it goes out before the
-          // wait for K, which frees its V slot for the copies sooner
-          if (pend_v[0] >= 0 && !(ok = issue_pv(0))) break;
-          if (!(ok = mbar_wait(&M.ring_full[gk % NR], (gk / NR) & 1, abort))) break;
-          const int mk = U.umask[j];
-          users[gv % NR] = __popc(mk);
-          // Every pending P.V goes out now, also for a slot that skips this
-          // block: a deferred P.V would pin its V tile in the ring.
+          // wait for K, which frees its V slot for the copies sooner.  Every
+          // pending P.V goes out in this step, also for a slot idle in it: a
+          // deferred P.V would pin its V tile in the ring.
 #pragma unroll
           for (int s = 0; s < 2; ++s) {
             if (ok && pend_v[s] >= 0) ok = issue_pv(s);
-            if (!ok || !((mk >> s) & 1)) continue;
+            if (!ok || blk[s] == kNoBlock) continue;
+            const uint32_t k = gk[s];
+            if (!(ok = mbar_wait(&M.ring_full[k % NR], (k / NR) & 1, abort, lim))) break;
             tc_fence_after();
-            const uint64_t dq = dq0[s], dk = dr_base + (uint64_t)(gk % NR) * (TILE >> 4);
+            const uint64_t dq = dq0[s], dk = dr_base + (uint64_t)(k % NR) * (TILE >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
               mma_ss(tm + s_col(s), dq + kstep_k_sw128(BM, kk), dk + kstep_k_sw128(BN, kk), idesc_s,
                      kk > 0 ? 1u : 0u);
             mma_commit(&M.s_full[s]);
-            pend_v[s] = (int)gv;
+            if (last[s]) mma_commit(&M.ring_empty[k % NR]);
+            pend_v[s] = (int)gv[s];
+            rel_v[s] = last[s];
           }
-          if (ok) mma_commit(&M.ring_empty[gk % NR]);
         }
         // tile end, per slot as soon as its last P.V is out: q P_h into the
         // (now free) S columns; Q is then free for the next unit.  Then
         // O += rho'_q S_U with rho'_q read from tensor memory (written by the
         // softmax warps) and S_U from the gather.
-        if (!(ok = mbar_wait(&M.pt_full, u & 1, abort))) break;
+        if (!(ok = mbar_wait(&M.pt_full, u & 1, abort, lim))) break;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           if (ok && pend_v[s] >= 0) ok = issue_pv(s);
@@ -759,8 +840,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           if (!ok || !U.active[s]) continue;
-          if (!(ok = mbar_wait(&M.lin_ready[s], uc[s] & 1, abort))) continue;
-          if (!(ok = mbar_wait(&M.zu_ready[s], uc[s] & 1, abort))) continue;
+          if (!(ok = mbar_wait(&M.lin_ready[s], uc[s] & 1, abort, lim))) continue;
+          if (!(ok = mbar_wait(&M.zu_ready[s], uc[s] & 1, abort, lim))) continue;
           tc_fence_after();
           const uint32_t suh = sAcc + s * (R * D * 4), sul = suh + Ly::SU_BYTES;
           const uint32_t a_hi = tm + s_col(s) + 32, a_lo = a_hi + R / 2;
@@ -831,8 +912,13 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
                                  const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                  const float* S_blk, const float* z_blk, const float* S_glb,
                                  const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
+                                 const int32_t* kb_h, uint64_t wait_ns, float* lse, float* den,
                                  cudaStream_t cs) {
   pairk::Params prm{};
+  prm.wait_ns = wait_ns;
+  prm.kb_h = kb_h;
+  prm.lse = lse;
+  prm.den = den;
   prm.B = s->B;
   prm.H = s->H;
   prm.N = s->N;

@@ -66,9 +66,22 @@ ROLA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Upper bound on one wait, in %globaltimer nanoseconds (1 s): far above any
-// legitimate wait inside one kernel, short enough that a broken pipeline
-// returns control instead of hanging the device.
+// Non-blocking test of the phase with `parity`.
+ROLA_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Default upper bound on one wait, in %globaltimer nanoseconds (1 s): far
+// above any legitimate wait inside one kernel, short enough that a broken
+// pipeline returns control instead of hanging the device.  The attention
+// kernels take the bound of their pipeline waits as a launch parameter; the
+// waits that drain copies and MMAs before a CTA exits always use this one.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 ROLA_DEV uint64_t globaltimer() {
@@ -78,8 +91,16 @@ ROLA_DEV uint64_t globaltimer() {
 }
 
 // Wait for the phase with `parity` to complete.  Returns false (and sets
-// *abort) if the limit ran out or another role already aborted.
-ROLA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// *abort) if `limit_ns` ran out or another role already aborted.  With
+// limit_ns == 0 the wait gives up as soon as it finds the phase incomplete
+// (a non-blocking test), which lets a caller exercise the abort path.
+ROLA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                        uint64_t limit_ns = kWaitLimitNs) {
+  if (limit_ns == 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    *abort = 1;
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t spins = 0;
@@ -87,7 +108,7 @@ ROLA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     if (++spins > 64) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }
@@ -358,31 +379,6 @@ ROLA_DEV float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^y for two lanes on the FMA pipe (offloads the special-function unit).
-// Range reduction: y = n + f with n = rint(y) taken from y + 1.5 * 2^23
-// (round to nearest) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
-// fitted here to 2^f in relative error on [-1/2, 1/2] (max relative error
-// 7.5e-5 in float32); 2^n applied by adding n to the exponent field.  y is
-// clamped below at -126 (results there are below 2^-125 and negligible).
-constexpr float kExp2C0 = 0.99992806f, kExp2C1 = 0.69326097f, kExp2C2 = 0.24261113f,
-                kExp2C3 = 0.055171624f;
-ROLA_DEV void exp2_poly2(float y0, float y1, float& e0, float& e1) {
-  const uint64_t shift = f32x2(12582912.f, 12582912.f);
-  const uint64_t nshift = f32x2(-12582912.f, -12582912.f);
-  const uint64_t y = f32x2(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
-  const uint64_t t = fadd2(y, shift);           // low bits hold rint(y)
-  const uint64_t n = fadd2(t, nshift);          // rint(y) as float
-  const uint64_t fr = ffma2(n, f32x2(-1.f, -1.f), y);
-  uint64_t p = ffma2(fr, f32x2(kExp2C3, kExp2C3), f32x2(kExp2C2, kExp2C2));
-  p = ffma2(p, fr, f32x2(kExp2C1, kExp2C1));
-  p = ffma2(p, fr, f32x2(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  f32x2_split(p, p0, p1);
-  f32x2_split(t, t0, t1);
-  e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // ---------------------------------------------------------------- misc

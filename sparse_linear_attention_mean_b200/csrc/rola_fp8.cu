@@ -133,3 +133,51 @@ extern "C" rola_status_t fp8_linear_w8a8(int32_t M, int32_t N, int32_t K, const 
   if (st != ROLA_OK) return st;
   return fp8_gemm_w8a8(M, N, K, xq, xs, w_q, w_scale, y, dev_err, stream);
 }
+
+// ---------------------------------------------------------------- FFN
+// Workspace of fp8_ffn_w8a8: codes and scales of x, the bf16 hidden
+// activation, and its codes and scales.
+struct FfnWs {
+  size_t xq, xs, h, hq, hs, total;
+};
+static FfnWs ffn_ws(int32_t M, int32_t D, int32_t F) {
+  using rola_internal::round_up;
+  FfnWs w{};
+  size_t off = 0;
+  w.xq = off; off += round_up((size_t)M * D, 256);
+  w.xs = off; off += round_up((size_t)M * 4, 256);
+  w.h = off;  off += round_up((size_t)M * F * 2, 256);
+  w.hq = off; off += round_up((size_t)M * F, 256);
+  w.hs = off; off += round_up((size_t)M * 4, 256);
+  w.total = off;
+  return w;
+}
+
+extern "C" size_t fp8_ffn_workspace_bytes(int32_t M, int32_t D, int32_t F) {
+  if (M < 1 || D < 1 || F < 1) return 0;
+  return ffn_ws(M, D, F).total;
+}
+
+extern "C" rola_status_t fp8_ffn_w8a8(int32_t M, int32_t D, int32_t F, const uint16_t* x,
+                                      const uint8_t* w1_q, const float* w1_scale,
+                                      const uint8_t* w2_q, const float* w2_scale, uint16_t* y,
+                                      void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
+  if (M < 1 || D < 1 || F < 1 || !x || !w1_q || !w1_scale || !w2_q || !w2_scale || !y)
+    return ROLA_ERR_INVALID_ARG;
+  if (D % 32 != 0 || F % 32 != 0) return ROLA_ERR_INVALID_ARG;
+  const FfnWs L = ffn_ws(M, D, F);
+  if (!ws || ws_bytes < L.total || !rola_host::aligned(ws, 256)) return ROLA_ERR_WORKSPACE;
+  char* base = reinterpret_cast<char*>(ws);
+  uint8_t* xq = reinterpret_cast<uint8_t*>(base + L.xq);
+  float* xs = reinterpret_cast<float*>(base + L.xs);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
+  uint8_t* hq = reinterpret_cast<uint8_t*>(base + L.hq);
+  float* hs = reinterpret_cast<float*>(base + L.hs);
+  rola_status_t st = fp8_quantize_rows_bf16(M, D, x, xq, xs, stream);
+  if (st != ROLA_OK) return st;
+  st = fp8_gemm_w8a8_act(M, F, D, xq, xs, w1_q, w1_scale, ROLA_ACT_GELU_TANH, h, dev_err, stream);
+  if (st != ROLA_OK) return st;
+  st = fp8_quantize_rows_bf16(M, F, h, hq, hs, stream);
+  if (st != ROLA_OK) return st;
+  return fp8_gemm_w8a8(M, D, F, hq, hs, w2_q, w2_scale, y, dev_err, stream);
+}

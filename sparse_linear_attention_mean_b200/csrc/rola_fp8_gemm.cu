@@ -14,7 +14,8 @@
 //               two 256-column accumulators so that the epilogue of one tile
 //               overlaps the main loop of the next;
 //   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, scale by
-//               x_scale[m] * w_scale[n], round to bf16, store.
+//               x_scale[m] * w_scale[n], optionally apply GELU (tanh form,
+//               the FFN's up projection), round to bf16, store.
 // Tiles are walked n-fastest so that the CTAs resident at one time share a
 // few 128-row panels of x_q in L2 while all of w_q stays L2-resident.
 // Every wait is bounded; on a timeout the CTA drains its copies and MMAs,
@@ -46,7 +47,15 @@ struct Params {
   const float* w_scale;
   uint16_t* y;
   int32_t* dev_err;
+  int act;  // ROLA_ACT_NONE or ROLA_ACT_GELU_TANH
 };
+
+// GELU in its tanh form, 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))), in
+// float32 with the CUDA math library's tanhf.
+ROLA_DEV float gelu_tanh(float u) {
+  const float kC = 0.7978845608028654f;  // sqrt(2 / pi)
+  return 0.5f * u * (1.f + tanhf(kC * fmaf(0.044715f * u, u * u, u)));
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -176,6 +185,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (m < p.M) {
           uint4* dst = reinterpret_cast<uint4*>(p.y + (size_t)m * p.N + n);
+          if (p.act == ROLA_ACT_GELU_TANH) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              r[j] = __float_as_uint(gelu_tanh(__uint_as_float(r[j]) * wsc[j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) wsc[j] = 1.f;
+          }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint4 o;
@@ -216,12 +232,13 @@ static bool make_fp8_map(CUtensorMap* m, const void* base, int rows, int K, int 
 }  // namespace fp8g
 }  // namespace rola
 
-extern "C" rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
-                                       const float* x_scale, const uint8_t* w_q,
-                                       const float* w_scale, uint16_t* y, int32_t* dev_err,
-                                       void* stream) {
+extern "C" rola_status_t fp8_gemm_w8a8_act(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
+                                           const float* x_scale, const uint8_t* w_q,
+                                           const float* w_scale, int32_t act, uint16_t* y,
+                                           int32_t* dev_err, void* stream) {
   using namespace rola::fp8g;
   if (M < 1 || N < 32 || K < 16 || N % 32 != 0 || K % 16 != 0) return ROLA_ERR_INVALID_ARG;
+  if (act != ROLA_ACT_NONE && act != ROLA_ACT_GELU_TANH) return ROLA_ERR_INVALID_ARG;
   if (!x_q || !x_scale || !w_q || !w_scale || !y) return ROLA_ERR_INVALID_ARG;
   if (!rola_host::aligned(x_q, 16) || !rola_host::aligned(w_q, 16) || !rola_host::aligned(y, 16) ||
       !rola_host::aligned(w_scale, 16) || !rola_host::aligned(x_scale, 4))
@@ -241,6 +258,7 @@ extern "C" rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const ui
   prm.w_scale = w_scale;
   prm.y = y;
   prm.dev_err = dev_err;
+  prm.act = act;
   if (cudaFuncSetAttribute(fp8_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem) !=
       cudaSuccess)
     return ROLA_ERR_CUDA;
@@ -248,4 +266,11 @@ extern "C" rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const ui
   const int grid = prm.tiles < nsm ? prm.tiles : nsm;
   fp8_gemm_kernel<<<grid, kThreads, kSmem, reinterpret_cast<cudaStream_t>(stream)>>>(ma, mb, prm);
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
+}
+
+extern "C" rola_status_t fp8_gemm_w8a8(int32_t M, int32_t N, int32_t K, const uint8_t* x_q,
+                                       const float* x_scale, const uint8_t* w_q,
+                                       const float* w_scale, uint16_t* y, int32_t* dev_err,
+                                       void* stream) {
+  return fp8_gemm_w8a8_act(M, N, K, x_q, x_scale, w_q, w_scale, ROLA_ACT_NONE, y, dev_err, stream);
 }

@@ -10,8 +10,6 @@
 #include <float.h>
 #include <math.h>
 
-#include <mutex>
-
 #include "rola_common.cuh"
 #include "rola_internal.h"
 
@@ -168,7 +166,10 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
 // ---------------------------------------------------------------- top-k
 // One warp per (b, h, query block).  Lane l holds the scores of blocks l,
 // l + 32, ... (MAXP per lane, n_blocks <= 32 * MAXP).  Order: score
-// descending, then block index ascending.
+// descending, then block index ascending.  A row keeps kb blocks, or
+// kb_h[h] of them when per-head counts are given (the row stride stays kb;
+// entries past the head's count are set to -1; a count outside [1, kb] is
+// clamped into it and reported as ROLA_DEVERR_BAD_INDEX).
 //
 // Fast path (k_b <= 32, k_b < n_blocks): the k_b-th largest of the 32 lane
 // maxima, T, is a lower bound of the k_b-th largest score (k_b lanes hold a
@@ -184,7 +185,9 @@ constexpr int kTopkWarps = 8;
 template <int MAXP>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const double* __restrict__ sigma,
                                                                int32_t* __restrict__ idx, int rows,
-                                                               int nb, int kb) {
+                                                               int nb, int kb_max,
+                                                               const int32_t* __restrict__ kb_h, int H,
+                                                               int32_t* dev_err) {
   __shared__ double cand_v[kTopkWarps][kCandCap];
   __shared__ int cand_j[kTopkWarps][kCandCap];
   __shared__ uint32_t kept_bits[kTopkWarps][32];
@@ -192,7 +195,14 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const double* __r
   const int warp = blockIdx.x * kTopkWarps + wib;
   if (warp >= rows) return;  // uniform per warp
   const double* s = sigma + (size_t)warp * nb;
-  int32_t* out = idx + (size_t)warp * kb;
+  int32_t* out = idx + (size_t)warp * kb_max;
+  int kb = kb_max;
+  if (kb_h) {
+    const int want = kb_h[(warp / nb) % H];
+    kb = min(max(want, 1), kb_max);
+    if (kb != want && lane == 0 && dev_err) atomicOr(dev_err, ROLA_DEVERR_BAD_INDEX);
+    for (int e = kb + lane; e < kb_max; e += 32) out[e] = -1;
+  }
   double v[MAXP];
 #pragma unroll
   for (int i = 0; i < MAXP; ++i) {
@@ -302,14 +312,17 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const double* __r
 }
 
 template <int MAXP>
-static void launch_topk(const double* sigma, int32_t* idx, int rows, int nb, int kb, cudaStream_t cs) {
-  topk_kernel<MAXP><<<(rows + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, cs>>>(sigma, idx, rows,
-                                                                                      nb, kb);
+static void launch_topk(const double* sigma, int32_t* idx, int rows, int nb, int kb, const int32_t* kb_h,
+                        int H, int32_t* dev_err, cudaStream_t cs) {
+  topk_kernel<MAXP><<<(rows + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, cs>>>(
+      sigma, idx, rows, nb, kb, kb_h, H, dev_err);
 }
 
-// Scores and top-k from pooled block means (float64 [B, H, nb, d]).
+// Scores and top-k from pooled block means (float64 [B, H, nb, d]); kb_h:
+// optional per-head kept counts (device int32 [H]).
 rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, const double* kbar,
-                                 double* sigma, int32_t* idx, cudaStream_t cs) {
+                                 double* sigma, int32_t* idx, cudaStream_t cs, const int32_t* kb_h,
+                                 int32_t* dev_err) {
   const int nb = rola_num_blocks(s);
   const int tiles = (nb + kScTile - 1) / kScTile;
   if (cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScSmemBytes) !=
@@ -318,12 +331,13 @@ rola_status_t select_from_pooled(const rola_shape_t* s, const double* qbar, cons
   score_kernel<<<dim3(tiles, tiles, s->B * s->H), 128, kScSmemBytes, cs>>>(qbar, kbar, sigma, s->H, s->d, nb);
   const int rows = s->B * s->H * nb;
   const int nper = (nb + 31) / 32;
-  if (nper <= 4) launch_topk<4>(sigma, idx, rows, nb, s->k_b, cs);
-  else if (nper <= 8) launch_topk<8>(sigma, idx, rows, nb, s->k_b, cs);
-  else if (nper <= 16) launch_topk<16>(sigma, idx, rows, nb, s->k_b, cs);
-  else if (nper <= 20) launch_topk<20>(sigma, idx, rows, nb, s->k_b, cs);
-  else if (nper <= 24) launch_topk<24>(sigma, idx, rows, nb, s->k_b, cs);
-  else launch_topk<kMaxPerLane>(sigma, idx, rows, nb, s->k_b, cs);
+  const int H = s->H, kb = s->k_b;
+  if (nper <= 4) launch_topk<4>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
+  else if (nper <= 8) launch_topk<8>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
+  else if (nper <= 16) launch_topk<16>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
+  else if (nper <= 20) launch_topk<20>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
+  else if (nper <= 24) launch_topk<24>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
+  else launch_topk<kMaxPerLane>(sigma, idx, rows, nb, kb, kb_h, H, dev_err, cs);
   return cudaGetLastError() == cudaSuccess ? ROLA_OK : ROLA_ERR_CUDA;
 }
 
@@ -344,6 +358,12 @@ extern "C" size_t rola_workspace_bytes(const rola_shape_t* s) { return rola_sele
 extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_t* q,
                                             const uint16_t* k, int32_t* idx, double* scores_opt,
                                             void* ws, size_t ws_bytes, void* stream) {
+  return select_blocks_impl(s, nullptr, q, k, idx, scores_opt, ws, ws_bytes, nullptr, stream);
+}
+
+rola_status_t rola::select_blocks_impl(const rola_shape_t* s, const int32_t* kb_h, const uint16_t* q,
+                                       const uint16_t* k, int32_t* idx, double* scores_opt, void* ws,
+                                       size_t ws_bytes, int32_t* dev_err, void* stream) {
   rola_status_t st = rola_internal::check_shape(s);
   if (st != ROLA_OK) return st;
   if (!q || !k || !idx) return ROLA_ERR_INVALID_ARG;
@@ -364,7 +384,7 @@ extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_
 
   pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
   if (cudaGetLastError() != cudaSuccess) return ROLA_ERR_CUDA;
-  return select_from_pooled(s, qbar, kbar, sig, idx, cs);
+  return select_from_pooled(s, qbar, kbar, sig, idx, cs, kb_h, dev_err);
 }
 
 // ---------------------------------------------------------------- selector without a workspace
@@ -374,31 +394,26 @@ extern "C" rola_status_t rola_select_blocks(const rola_shape_t* s, const uint16_
 // call site: a host-side plugin or language binding that holds only the q, k
 // and idx buffers and has no device allocator of its own.  Nothing is
 // allocated per call: the array exists once per device for the life of the
-// context, and its address is looked up (cudaGetSymbolAddress) on the first
-// call on each device -- so that first call does set-up work and should come
-// before any stream capture.  Every scratch word is written before it is
-// read, so nothing needs clearing between calls; calls that overlap in time
-// on one device (several streams or host threads) share the array and race.
+// context.  In host code the array's name is only a stand-in, so every call
+// asks the runtime for its device address on the current device
+// (cudaGetSymbolAddress).  That lookup is cheap once the library's module is
+// loaded on the device; the first call on a device loads it, so that first
+// call should come before any stream capture.  Asking on every call (instead
+// of caching the address) keeps the entry point correct after a device reset
+// or a re-created primary context, where the array has a new address.  Every
+// scratch word is written before it is read, so nothing needs clearing
+// between calls; calls that overlap in time on one device (several streams or
+// host threads) share the array and race.
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
 static __device__ __align__(256) unsigned char g_select_scratch[kNoAllocScratchBytes];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices];
-std::mutex g_scratch_mu;
-
 // Device address of the scratch array on the current device, or null.
 void* scratch_on_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = p;
-  }
-  return g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace
@@ -423,5 +438,5 @@ extern "C" rola_status_t rola_select_blocks_noalloc(const rola_shape_t* s, const
       ws + rola_internal::round_up(2 * (size_t)s->B * s->H * nb * s->d * sizeof(double), 256));
   pool_kernel<<<dim3(nb, s->B, 2), 256, 0, cs>>>(q, k, qbar, kbar, s->N, s->H, s->d, s->block, nb);
   if (cudaGetLastError() != cudaSuccess) return ROLA_ERR_CUDA;
-  return select_from_pooled(s, qbar, kbar, sig, idx, cs);
+  return select_from_pooled(s, qbar, kbar, sig, idx, cs, nullptr, nullptr);
 }

@@ -24,7 +24,8 @@ Input recipe (the pages give none, so this is a stated choice):
   the tiny workload, ``U(0.2, 1)`` per head otherwise.
 * Everything is rounded float64 -> float32 -> bfloat16 (round to nearest even).
 * The full-block workload adds ``x ~ N(0, 1)`` ``[N, 5120]`` and four
-  ``5120 x 5120`` float32 weights ``~ N(0, 1/5120)``.
+  ``5120 x 5120`` float32 weights ``~ N(0, 1/5120)``; its FFN weights are
+  ``W1 [13824, 5120] ~ N(0, 1/5120)`` and ``W2 [5120, 13824] ~ N(0, 1/13824)``.
 
 Tokens are in frame-major raster order: token ``n`` sits at
 ``t = n // (Hg*W)``, ``y = (n // W) % Hg``, ``x = n % W``.
@@ -43,6 +44,11 @@ _CHUNK = 2048  # tokens per independently seeded noise chunk
 _S_FIELD, _S_PROJ, _S_GATE = 1, 2, 3
 _S_NOISE = {"q": 10, "k": 11, "v": 12}
 _S_X, _S_WQKV, _S_WO = 20, 21, 22
+_S_W1, _S_W2 = 23, 24
+
+# FFN hidden width of the 14B model (the pages give none; the Wan2.1-14B
+# transformer's feed-forward width is taken as the stated reading)
+FFN_HIDDEN_14B = 13824
 
 
 @dataclasses.dataclass(frozen=True)
@@ -226,6 +232,15 @@ def make_block_inputs(w: Workload, threads: int = 8) -> dict:
     Wo = (_rng(w.seed, _S_WO).standard_normal((D, D), dtype=np.float32) * np.float32(sd))
     return {"x": x, "Wq": Wqkv[:D], "Wk": Wqkv[D:2 * D], "Wv": Wqkv[2 * D:], "Wo": Wo,
             "P": make_projection(w), "gate": make_gate(w)}
+
+
+def make_ffn_weights(w: Workload, hidden: int = FFN_HIDDEN_14B) -> dict:
+    """float32 FFN weights of the full block: W1 [hidden, D] ~ N(0, 1/D) (up
+    projection) and W2 [D, hidden] ~ N(0, 1/hidden) (down projection)."""
+    D = w.model_dim
+    W1 = _rng(w.seed, _S_W1).standard_normal((hidden, D), dtype=np.float32) * np.float32(1.0 / math.sqrt(D))
+    W2 = _rng(w.seed, _S_W2).standard_normal((D, hidden), dtype=np.float32) * np.float32(1.0 / math.sqrt(hidden))
+    return {"W1": W1, "W2": W2}
 
 
 def make_uniform(shape, seed: int, lo: float, hi: float) -> np.ndarray:

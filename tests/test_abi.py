@@ -89,6 +89,20 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.fp8_quantize_rows_bf16(4, 15, ok, ok, ok, None) == 1                          # K % 16
 
 
+def test_bounded_attention_arguments_rejected_on_host(lib):
+    """The attention entry with an explicit wait bound checks its arguments
+    like the default one before any launch."""
+    cs = rb.Shape(1, 2, 64, 4, 16, 16, 64, 4, 16).c()
+    ok = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4097)
+    fn = lib.rola_attention_fwd_bounded
+    args = [ok] * 12
+    assert fn(ctypes.byref(cs), *args[:3], None, *args[4:], ctypes.c_uint64(0), None) == 1  # null idx
+    assert fn(ctypes.byref(cs), odd, *args[1:], ctypes.c_uint64(0), None) == 5               # misaligned q
+    bad = rb.Shape(1, 2, 64, 4, 16, 16, 64, 17, 16).c()                                      # k_b > n_blocks
+    assert fn(ctypes.byref(bad), *args, ctypes.c_uint64(10**9), None) == 1
+
+
 def test_fp8_gemm_arguments_rejected_on_host(lib):
     ok = ctypes.c_void_p(4096)
     odd = ctypes.c_void_p(4104)  # 8-byte aligned only
@@ -100,6 +114,17 @@ def test_fp8_gemm_arguments_rejected_on_host(lib):
     assert gemm(64, 64, 64, odd, ok, ok, ok, ok, None, None) == 5   # misaligned codes
     assert gemm(64, 64, 64, ok, ok, ok, odd, ok, None, None) == 5   # misaligned w_scale
     assert lib.fp8_linear_w8a8(64, 64, 64, ok, ok, ok, ok, None, 0, None, None) == 3  # no workspace
+    act = lib.fp8_gemm_w8a8_act
+    assert act(64, 64, 64, ok, ok, ok, ok, 2, ok, None, None) == 1       # unknown activation
+    assert act(64, 40, 64, ok, ok, ok, ok, 1, ok, None, None) == 1       # N % 32
+    ffn = lib.fp8_ffn_w8a8
+    assert ffn(64, 64, 96, ok, ok, ok, ok, ok, ok, None, 0, None, None) == 3    # no workspace
+    assert ffn(64, 64, 100, ok, ok, ok, ok, ok, ok, ok, 1 << 30, None, None) == 1  # F % 32
+    assert ffn(64, 64, 96, ok, ok, ok, None, ok, ok, ok, 1 << 30, None, None) == 1  # null w2
+    r256 = lambda n: -(-n // 256) * 256
+    M, D, F = 75600, 5120, 13824
+    assert lib.fp8_ffn_workspace_bytes(M, D, F) == (r256(M * D) + r256(4 * M) + r256(2 * M * F)
+                                                    + r256(M * F) + r256(4 * M))
 
 
 def test_timed_layer_event_count_checked_on_host(lib):
@@ -136,3 +161,5 @@ def test_binding_constants_match_the_header():
     defines = dict(re.findall(r"#define\s+ROLA_DEVERR_(\w+)\s+(0x[0-9a-fA-F]+)", text))
     assert int(defines["BAD_INDEX"], 16) == rb.DEVERR_BAD_INDEX
     assert int(defines["TIMEOUT"], 16) == rb.DEVERR_TIMEOUT
+    acts = dict(re.findall(r"#define\s+ROLA_ACT_(\w+)\s+(\d+)", text))
+    assert int(acts["NONE"]) == rb.ACT_NONE and int(acts["GELU_TANH"]) == rb.ACT_GELU_TANH

@@ -90,6 +90,27 @@ def test_gemm_small(M, N, K):
     _check_gemm(y, fo.gemm_w8a8(xq, xs, wq, ws), f"gemm {M}x{N}x{K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(200, 96, 80), (333, 544, 2064), (1000, 768, 1024)])
+def test_gemm_gelu_small(M, N, K):
+    """The GELU epilogue (the FFN's up projection): y = bf16(gelu(product))."""
+    xq = _random_codes((M, K), 21 + M)
+    wq = _random_codes((N, K), 23 + N)
+    g = np.random.default_rng(M * N + K)
+    # scales that put the products in GELU's curved range (|u| up to ~6)
+    ones_m, ones_n = np.ones(M, np.float32), np.ones(N, np.float32)
+    raw = np.abs(fo.gemm_w8a8(xq, ones_m, wq, ones_n)).max(axis=1)
+    xs = (6.0 / np.maximum(raw, 1.0) * g.uniform(0.3, 1.0, size=M)).astype(np.float32)
+    ws = g.uniform(0.5, 1.0, size=N).astype(np.float32)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = rb.fp8_gemm(torch.from_numpy(xq).cuda(), torch.from_numpy(xs).cuda(), torch.from_numpy(wq).cuda(),
+                    torch.from_numpy(ws).cuda(), dev_err=err, act=rb.ACT_GELU_TANH)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    prod = fo.gemm_w8a8(xq, xs, wq, ws)
+    assert np.abs(prod).max() > 2.0 and (prod < -0.5).mean() > 0.02
+    _check_gemm(y, fo.gelu_tanh(prod), f"gemm+gelu {M}x{N}x{K}")
+
+
 def test_gemm_rejects_bad_shapes():
     xq = torch.zeros((4, 64), dtype=torch.uint8, device="cuda")
     xs = torch.ones(4, device="cuda")
@@ -213,4 +234,67 @@ def test_attention_block_chain():
         for a, rows in r.o.items():
             lo, hi = ro.block_range(a, w.block, w.N)
             check_close(o64[b, lo:hi, heads[j], :], rows, what=f"head {heads[j]} block {a}")
-    assert torch.isfinite(y.float()).all()
+    # the output projection on sampled rows: the oracle's W8A8 product of the
+    # GPU's attention output (its own quantisation of those rows and of W_o)
+    M = w.B * w.N
+    rows = np.unique(np.concatenate([np.arange(0, 4), np.arange(M - 80, M, 19), [M - 1],
+                                     np.random.default_rng(8).integers(0, M, 24)]))
+    o_rows = o.view(M, D)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    w_codes, w_scale = fo.quantize_rows(np.ascontiguousarray(inp["Wo"]))
+    assert np.array_equal(wo_q.cpu().numpy(), w_codes)
+    ref_y = fo.linear_w8a8(o_rows, w_codes, w_scale)
+    _check_gemm(y[torch.from_numpy(rows).cuda()], ref_y, "output projection 75600x5120x5120")
+
+
+def test_ffn_full_size_sampled():
+    """The full 14B-720P FFN in W8A8 (x [75600, 5120] -> GELU(x W1^T) [75600,
+    13824] -> [75600, 5120]), the benchmark's launch configuration.  The fused
+    entry equals the step-by-step chain bit for bit; on sampled rows the hidden
+    activation matches the oracle's GELU of the W8A8 product, and the output
+    matches the oracle's W8A8 product of the GPU's hidden activation (its own
+    quantisation of those rows)."""
+    w, inp = _block_inputs()
+    ffw = synth.make_ffn_weights(w)
+    M, D, F = w.B * w.N, w.model_dim, ffw["W1"].shape[0]
+    x = _bf16_dev(inp["x"])
+    w1q, w1s = rb.fp8_quantize_weight(torch.from_numpy(ffw["W1"]).cuda())
+    w2q, w2s = rb.fp8_quantize_weight(torch.from_numpy(ffw["W2"]).cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = rb.fp8_ffn(x, w1q, w1s, w2q, w2s, dev_err=err)
+    xq, xsc = rb.fp8_quantize_rows(x)
+    h = rb.fp8_gemm(xq, xsc, w1q, w1s, dev_err=err, act=rb.ACT_GELU_TANH)
+    hq, hsc = rb.fp8_quantize_rows(h)
+    y2 = rb.fp8_gemm(hq, hsc, w2q, w2s, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(y, y2)
+    rows = np.unique(np.concatenate([np.arange(0, 4), np.arange(M - 80, M, 19), [M - 1],
+                                     np.random.default_rng(9).integers(0, M, 24)]))
+    rows_d = torch.from_numpy(rows).cuda()
+    w1_codes, w1_scale = fo.quantize_rows(ffw["W1"])
+    w2_codes, w2_scale = fo.quantize_rows(ffw["W2"])
+    assert np.array_equal(w1q.cpu().numpy(), w1_codes) and np.array_equal(w2q.cpu().numpy(), w2_codes)
+    x_codes, x_scale = fo.quantize_rows(_bf16_f32(inp["x"][rows]))
+    h_ref = fo.gelu_tanh(fo.gemm_w8a8(x_codes, x_scale, w1_codes, w1_scale))
+    _check_gemm(h[rows_d], h_ref, "FFN up projection + GELU 75600x13824x5120")
+    h_rows = h[rows_d].float().cpu().numpy()
+    y_ref = fo.linear_w8a8(h_rows, w2_codes, w2_scale)
+    _check_gemm(y[rows_d], y_ref, "FFN down projection 75600x5120x13824")
+
+
+def test_ffn_small_matches_oracle_chain():
+    """A small ragged FFN through the fused entry against the oracle's whole
+    chain (its own quantisation, GELU and bf16 hidden activation)."""
+    g = np.random.default_rng(12)
+    M, D, F = 300, 256, 608
+    x_bits = synth.make_normal_bf16((M, D), seed=12, stream=3, std=1.0)
+    W1 = (g.standard_normal((F, D)) / np.sqrt(D)).astype(np.float32)
+    W2 = (g.standard_normal((D, F)) / np.sqrt(F)).astype(np.float32)
+    w1q, w1s = rb.fp8_quantize_weight(torch.from_numpy(W1).cuda())
+    w2q, w2s = rb.fp8_quantize_weight(torch.from_numpy(W2).cuda())
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = rb.fp8_ffn(_bf16_dev(x_bits), w1q, w1s, w2q, w2s, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    _, y_ref = fo.ffn_w8a8(_bf16_f32(x_bits), *fo.quantize_rows(W1), *fo.quantize_rows(W2))
+    _check_gemm(y, y_ref, "FFN 300x256x608")

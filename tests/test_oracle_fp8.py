@@ -91,3 +91,57 @@ def test_gemm_exact_on_representable_operands():
     qb, sb = fo.quantize_rows(b.astype(np.float32))
     assert np.all(sa == 1.0) and np.all(sb == 1.0)
     np.testing.assert_array_equal(fo.gemm_w8a8(qa, sa, qb, sb), a @ b.T)
+
+
+def test_round_bf16_matches_torch():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(100000) * 10.0 ** rng.integers(-6, 6, 100000),
+                        [0.0, -0.0, 1.0, 1.00390625, 1.005859375, 3.0e38]])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(fo.round_bf16(x.astype(np.float32).astype(np.float64)), want)
+    # ties between bf16 neighbours go to the even mantissa
+    assert fo.round_bf16(np.array([1.00390625]))[0] == 1.0          # 1 + 2^-8: tie, 1.0 is even
+    assert fo.round_bf16(np.array([1.01171875]))[0] == 1.015625     # 1 + 3*2^-8: tie, up to even
+
+
+def test_gelu_tanh_matches_torch_and_limits():
+    u = np.linspace(-12.0, 12.0, 4001)
+    want = torch.nn.functional.gelu(torch.from_numpy(u), approximate="tanh").numpy()
+    np.testing.assert_allclose(fo.gelu_tanh(u), want, rtol=1e-13, atol=1e-15)
+    assert fo.gelu_tanh(np.array([0.0]))[0] == 0.0
+    big = np.array([30.0, -30.0])
+    np.testing.assert_allclose(fo.gelu_tanh(big), [30.0, 0.0], atol=1e-300)
+    # GELU is not odd: gelu(u) - gelu(-u) = u
+    np.testing.assert_allclose(fo.gelu_tanh(u) - fo.gelu_tanh(-u), u, atol=1e-12)
+
+
+def test_ffn_matches_an_independent_library_chain():
+    """The FFN composition against the same steps taken with torch's own
+    float8_e4m3fn casts, float64 matmuls, GELU and bfloat16 rounding: a wrong
+    step order (GELU after the bf16 rounding, a missing scale, the scales of
+    the wrong operand) fails it."""
+    rng = np.random.default_rng(4)
+    M, D, F = 24, 64, 96
+    x = (rng.standard_normal((M, D)) * 2).astype(np.float32)
+    W1 = (rng.standard_normal((F, D)) / 8).astype(np.float32)
+    W2 = (rng.standard_normal((D, F)) / 10).astype(np.float32)
+    c1, s1 = fo.quantize_rows(W1)
+    c2, s2 = fo.quantize_rows(W2)
+    h, y = fo.ffn_w8a8(x, c1, s1, c2, s2)
+
+    def tq(a):  # torch: per-row E4M3 quantisation, reciprocal and product in float32
+        a = torch.from_numpy(a)
+        amax = a.abs().amax(dim=1)
+        inv = (448.0 / amax).to(torch.float32)
+        q = (a * inv[:, None]).to(torch.float8_e4m3fn).to(torch.float64)
+        return q, (amax / 448.0).to(torch.float64)
+
+    qx, sx = tq(x)
+    qw1, sw1 = tq(W1)
+    qw2, sw2 = tq(W2)
+    hid = (qx @ qw1.T) * sx[:, None] * sw1[None, :]
+    ht = torch.nn.functional.gelu(hid, approximate="tanh").to(torch.bfloat16)
+    qh, sh = tq(ht.to(torch.float32).numpy())
+    yt = (qh @ qw2.T) * sh[:, None] * sw2[None, :]
+    np.testing.assert_array_equal(h, ht.to(torch.float64).numpy())
+    np.testing.assert_allclose(y, yt.numpy(), rtol=1e-12, atol=1e-12)

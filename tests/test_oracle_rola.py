@@ -297,3 +297,30 @@ def test_generator_is_deterministic_and_bf16():
     # structured q and k share the positional field: strongly correlated
     k = ro.bf16_to_f64(a["k"])
     assert np.corrcoef(q.ravel(), k.ravel())[0, 1] > 0.6
+
+
+def test_per_head_selection_is_nested_and_brute_force():
+    """Head-adaptive counts: each head's kept set is the brute-force top
+    kb_per_head[h] by (score desc, index asc), the unused entries are -1, and
+    the sets are nested in the count (keeping one more block adds one)."""
+    rng = np.random.default_rng(21)
+    B, N, H, d, bs = 1, 160, 3, 8, 16
+    inp = {"q": (rng.standard_normal((B, N, H, d)) * 4).astype(np.float32),
+           "k": (rng.standard_normal((B, N, H, d)) * 4).astype(np.float32)}
+    # bf16 bit patterns of the draws (truncated: any bf16 values will do here)
+    inp = {kk: (vv.view(np.uint32) >> 16).astype(np.uint16) for kk, vv in inp.items()}
+    kbh = [1, 4, 7]
+    idx, sig = ro.select_all_per_head(inp, bs, kbh, 7)
+    nb = N // bs
+    for h, kh in enumerate(kbh):
+        assert (idx[0, h, :, kh:] == -1).all()
+        for a in range(nb):
+            order = sorted(range(nb), key=lambda j: (-sig[0, h, a, j], j))
+            assert sorted(order[:kh]) == idx[0, h, a, :kh].tolist()
+    for kh in range(1, nb):
+        small, _ = ro.select_all_per_head(inp, bs, [kh] * H, nb)
+        big, _ = ro.select_all_per_head(inp, bs, [kh + 1] * H, nb)
+        for h in range(H):
+            for a in range(nb):
+                s1, s2 = set(small[0, h, a, :kh].tolist()), set(big[0, h, a, :kh + 1].tolist())
+                assert s1 < s2 and len(s2 - s1) == 1
