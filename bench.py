@@ -278,7 +278,9 @@ def run_gpu(args) -> int:
     assert int(layer.dev_err.item()) == 0
     reuse_ms = statistics.mean(e[0].elapsed_time(e[4]) for e in ev_r)
     reuse = {"ms_per_layer": reuse_ms, "tflops": flop / (reuse_ms * 1e-3) / 1e12,
-             "selection_skipped_ms": statistics.mean(per_stage["score+topk"]) if "score+topk" in per_stage else None}
+             "stages_ms": {nm: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev_r)
+                           for i, nm in enumerate(stage_names)},
+             "selection_ms_when_selecting": statistics.mean(per_stage["score+topk"])}
 
     # one FP8 W8A8 projection of the full attention block (x [N, 5120] ->
     # [N, 5120]: quantisation + tcgen05 GEMM), timed on its own after the layer

@@ -201,7 +201,10 @@ rola_status_t rola_attention_fwd_bounded(const rola_shape_t* shape, const uint16
 /* ---------------------------------------------------------------- backward */
 
 /* rola_attention_fwd (d = 128, 128-token blocks, k_b <= 256, n_blocks <= 1024)
- * that also saves, per row, what rola_attention_bwd reads:
+ * that also saves what rola_attention_bwd reads:
+ *   out_lo  bf16 [B, N, H, d]: the output's rounding residual, bf16(o - out)
+ *        with o the float32 result (out + out_lo carries ~16 mantissa bits,
+ *        which the backward's D = dout . o_sp needs);
  *   lse  float [B, H, N]: natural log of sum over the kept valid keys of
  *        exp(q . k / sqrt(d)) (-inf for a row without kept blocks);
  *   den  float [B, H, N]: the linear branch's denominator psi_q . z_U (NaN
@@ -211,8 +214,9 @@ rola_status_t rola_attention_fwd_bounded(const rola_shape_t* shape, const uint16
 rola_status_t rola_attention_fwd_train(const rola_shape_t* shape, const uint16_t* q, const uint16_t* k,
                                        const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                        const float* S_blk, const float* z_blk, const float* S_glb,
-                                       const float* z_glb, const float* gate, uint16_t* out, float* lse,
-                                       float* den, int32_t* dev_err, void* stream);
+                                       const float* z_glb, const float* gate, uint16_t* out,
+                                       uint16_t* out_lo, float* lse, float* den, int32_t* dev_err,
+                                       void* stream);
 
 /* Workspace of rola_attention_bwd (256-byte aligned), 0 for an invalid or
  * unsupported shape. */
@@ -229,7 +233,7 @@ size_t rola_attention_bwd_workspace_bytes(const rola_shape_t* shape);
  * the block states S_b = sum rho_k v^T, z_b = sum psi_k, the rotary
  * rotation, the feature map elu + 1 and the projection P_h.
  *   q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate: the forward's inputs
- *   out, lse, den: its output and saved statistics (rola_attention_fwd_train)
+ *   out, out_lo, lse, den: its output and saved quantities (rola_attention_fwd_train)
  *   dout   bf16 [B, N, H, d], the gradient reaching out
  *   dq, dk, dv  out, bf16 [B, N, H, d] (padding rows not written)
  *   dP     out, float [H, d, r];   dgate  out, float [H]
@@ -243,7 +247,8 @@ rola_status_t rola_attention_bwd(const rola_shape_t* shape, const uint16_t* q, c
                                  const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                  const float* S_blk, const float* z_blk, const float* S_glb,
                                  const float* z_glb, const float* gate, const uint16_t* out,
-                                 const float* lse, const float* den, const uint16_t* dout, uint16_t* dq,
+                                 const uint16_t* out_lo, const float* lse, const float* den,
+                                 const uint16_t* dout, uint16_t* dq,
                                  uint16_t* dk, uint16_t* dv, float* dP, float* dgate, void* ws,
                                  size_t ws_bytes, int32_t* dev_err, void* stream);
 

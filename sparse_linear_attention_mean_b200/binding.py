@@ -120,11 +120,11 @@ def lib() -> ctypes.CDLL:
         L.rola_layer_fwd_ex.argtypes = [sp, ctypes.POINTER(LayerOpts), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                         vp, ctypes.POINTER(ctypes.c_void_p), i32]
         L.rola_attention_fwd_train.restype = ctypes.c_int
-        L.rola_attention_fwd_train.argtypes = [sp] + [vp] * 14 + [vp]
+        L.rola_attention_fwd_train.argtypes = [sp] + [vp] * 15 + [vp]
         L.rola_attention_bwd_workspace_bytes.restype = sz
         L.rola_attention_bwd_workspace_bytes.argtypes = [sp]
         L.rola_attention_bwd.restype = ctypes.c_int
-        L.rola_attention_bwd.argtypes = [sp] + [vp] * 19 + [vp, sz, vp, vp]
+        L.rola_attention_bwd.argtypes = [sp] + [vp] * 20 + [vp, sz, vp, vp]
         L.rola_layer_kernel_launches.restype = ctypes.c_int
         L.rola_layer_kernel_launches.argtypes = [sp]
         L.rola_layer_fwd_host.restype = ctypes.c_int
@@ -259,26 +259,28 @@ def attention_fwd(shape: Shape, q, k, v, idx, P, states, gate, *, out=None, dev_
 
 
 def attention_fwd_train(shape: Shape, q, k, v, idx, P, states, gate, *, dev_err=None, stream=None):
-    """Forward that also returns the statistics the backward reads:
-    (out bf16 [B, N, H, d], lse float [B, H, N], den float [B, H, N])."""
+    """Forward that also returns what the backward reads: (out, out_lo bf16
+    [B, N, H, d], lse float [B, H, N], den float [B, H, N])."""
     act = (shape.B, shape.N, shape.H, shape.d)
     S_blk, z_blk, S_glb, z_glb = states
     out = torch.empty(act, dtype=torch.bfloat16, device=q.device)
+    out_lo = torch.empty_like(out)
     lse = torch.empty((shape.B, shape.H, shape.N), dtype=torch.float32, device=q.device)
     den = torch.empty_like(lse)
     _check(lib().rola_attention_fwd_train(ctypes.byref(shape.c()), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(P),
                                           _ptr(S_blk), _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate),
-                                          _ptr(out), _ptr(lse), _ptr(den), _ptr(dev_err), _stream(stream)),
+                                          _ptr(out), _ptr(out_lo), _ptr(lse), _ptr(den), _ptr(dev_err),
+                                          _stream(stream)),
            "rola_attention_fwd_train")
-    return out, lse, den
+    return out, out_lo, lse, den
 
 
-def attention_bwd(shape: Shape, q, k, v, idx, P, states, gate, out, lse, den, dout, *, dev_err=None,
+def attention_bwd(shape: Shape, q, k, v, idx, P, states, gate, out, out_lo, lse, den, dout, *, dev_err=None,
                   stream=None, workspace=None):
     """Gradients (dq, dk, dv bf16 [B, N, H, d], dP float [H, d, r], dgate
     float [H]) of sum(dout * out) for the forward of attention_fwd_train."""
     act = (shape.B, shape.N, shape.H, shape.d)
-    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (out_lo, "out_lo"), (dout, "dout")):
         _need(t, torch.bfloat16, act, nm)
     S_blk, z_blk, S_glb, z_glb = states
     dq, dk, dv = (torch.zeros(act, dtype=torch.bfloat16, device=q.device) for _ in range(3))
@@ -291,8 +293,8 @@ def attention_bwd(shape: Shape, q, k, v, idx, P, states, gate, out, lse, den, do
     if workspace is None or workspace.numel() < nbytes:
         workspace = _ws(nbytes, q.device)
     _check(lib().rola_attention_bwd(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(P), _ptr(S_blk),
-                                    _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate), _ptr(out), _ptr(lse),
-                                    _ptr(den), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dP), _ptr(dgate),
+                                    _ptr(z_blk), _ptr(S_glb), _ptr(z_glb), _ptr(gate), _ptr(out), _ptr(out_lo),
+                                    _ptr(lse), _ptr(den), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dP), _ptr(dgate),
                                     _ptr(workspace), nbytes, _ptr(dev_err), _stream(stream)),
            "rola_attention_bwd")
     return dq, dk, dv, dP, dgate

@@ -600,7 +600,7 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
                                  const float* S_blk, const float* z_blk, const float* S_glb,
                                  const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
                                  const int32_t* kb_h, uint64_t wait_ns, float* lse, float* den,
-                                 cudaStream_t cs);
+                                 uint16_t* out_lo, cudaStream_t cs);
 
 }  // namespace rola
 
@@ -646,7 +646,7 @@ rola_status_t rola::attention_launch(const rola_shape_t* s, const int32_t* kb_h,
   if (pair_kernel_supports(s) && rola_host::aligned(S_blk, 32) && rola_host::aligned(S_glb, 32) &&
       rola_host::aligned(P, 16))
     return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, kb_h,
-                              wait_limit_ns, nullptr, nullptr, cs);
+                              wait_limit_ns, nullptr, nullptr, nullptr, cs);
   if (s->d == 128 && s->block == 128 && s->r == 32) return launch_attn<128, 128, 32>(s, q, k, v, prm, cs);
   if (s->d == 128 && s->block == 128 && s->r == 16) return launch_attn<128, 128, 16>(s, q, k, v, prm, cs);
   if (s->d == 64 && s->block == 64 && s->r == 16) return launch_attn<64, 64, 16>(s, q, k, v, prm, cs);
@@ -684,18 +684,19 @@ extern "C" rola_status_t rola_attention_fwd_train(const rola_shape_t* s, const u
                                                   const int32_t* idx, const uint16_t* P,
                                                   const float* S_blk, const float* z_blk,
                                                   const float* S_glb, const float* z_glb,
-                                                  const float* gate, uint16_t* out, float* lse,
-                                                  float* den, int32_t* dev_err, void* stream) {
+                                                  const float* gate, uint16_t* out, uint16_t* out_lo,
+                                                  float* lse, float* den, int32_t* dev_err, void* stream) {
   rola_status_t st = rola_internal::check_shape(s);
   if (st != ROLA_OK) return st;
-  if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out || !lse || !den)
+  if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out || !out_lo || !lse ||
+      !den)
     return ROLA_ERR_INVALID_ARG;
   if (!pair_kernel_supports(s)) return ROLA_ERR_UNSUPPORTED;
   if (!rola_host::aligned(q, 16) || !rola_host::aligned(k, 16) || !rola_host::aligned(v, 16) ||
       !rola_host::aligned(out, 16) || !rola_host::aligned(S_blk, 32) || !rola_host::aligned(S_glb, 32) ||
       !rola_host::aligned(idx, 4) || !rola_host::aligned(P, 16) || !rola_host::aligned(lse, 4) ||
-      !rola_host::aligned(den, 4))
+      !rola_host::aligned(den, 4) || !rola_host::aligned(out_lo, 16))
     return ROLA_ERR_ALIGNMENT;
   return launch_pair_kernel(s, q, k, v, idx, P, S_blk, z_blk, S_glb, z_glb, gate, out, dev_err, nullptr,
-                            kWaitLimitNs, lse, den, reinterpret_cast<cudaStream_t>(stream));
+                            kWaitLimitNs, lse, den, out_lo, reinterpret_cast<cudaStream_t>(stream));
 }

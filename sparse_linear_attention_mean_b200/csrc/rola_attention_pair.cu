@@ -131,6 +131,7 @@ struct Params {
   const int32_t* kb_h;  // per-head kept counts (NULL: kb for every head); idx rows keep stride kb
   float* lse;  // optional [B, H, N]: natural log-sum-exp of the scaled kept scores per row
   float* den;  // optional [B, H, N]: linear denominator psi_q . z_U (NaN when the complement is empty)
+  uint16_t* out_lo;  // optional [B, N, H, d]: bf16 of out (in fp32) minus its bf16 rounding
   RopeTable rope;
   // rotary table: entry of pair pr at position pos = tab_base[pr] + pos * tab_stride[pr];
   // pair pr fills entries [tab_first[pr], tab_first[pr + 1]) of the fill order
@@ -174,7 +175,10 @@ ROLA_DEV void decode_unit(const Params& p, int id, int& b, int& h, int& pair) {
   b = id / (p.npairs * p.H);
 }
 
-template <int R>
+// kLoP (the training forward): P enters P.V as bf16 hi + lo, so that the
+// output -- which the backward's D = dout . o_sp is formed from -- carries ~16
+// mantissa bits instead of the ~8 of bf16 P.
+template <int R, bool kLoP>
 __global__ void __launch_bounds__(kThreads, 1)
     rola_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -300,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint64_t nm2 = f32x2(-m, -m);
           uint64_t acc2 = f32x2(0.f, 0.f);
+          uint32_t lo8[8];  // kLoP: residuals of 16 columns, stored as they complete
 #pragma unroll
           for (int c = 0; c < 128; c += 2) {
             float y0, y1;
@@ -307,6 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
             acc2 = fadd2(acc2, f32x2(p0, p1));
             x[c >> 1] = pack_bf16(p0, p1);
+            if constexpr (kLoP) {
+              // P - bf16(P) over columns [64, 128) of the S buffer (the row is
+              // in registers; its tensor-memory copy is no longer read)
+              lo8[(c >> 1) & 7] = pack_bf16(p0 - bf16_lo(x[c >> 1]), p1 - bf16_hi(x[c >> 1]));
+              if (((c >> 1) & 7) == 7) tmem_st8(sc + Ly::P_OFF + 64 + ((c >> 1) & ~7), lo8);
+            }
           }
           // bf16 P over columns [0, 64) of the S buffer (S already read)
           tmem_st32_at<0>(sc + Ly::P_OFF, x);
@@ -414,6 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               orow[2 * c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
               orow[2 * c + 1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+            }
+            if (p.out_lo) {
+              // the bf16 rounding residual of the output (the backward's D needs ~16 bits)
+              uint32_t lv[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                lv[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv_l - bf16_lo(wv[e]),
+                                  __uint_as_float(o[2 * e + 1]) * inv_l - bf16_hi(wv[e]));
+              uint4* lrow = reinterpret_cast<uint4*>(p.out_lo + (((size_t)U.b * p.N + n) * p.H + U.h) * D);
+              lrow[2 * c] = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+              lrow[2 * c + 1] = make_uint4(lv[4], lv[5], lv[6], lv[7]);
             }
           }
         }
@@ -770,9 +792,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dv = dv_base + (uint64_t)(gv % NR) * (TILE >> 4);
           const uint32_t acc0 = first_pv[s] ? 0u : 1u;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
+          for (int kk = 0; kk < BN / 16; ++kk) {
             mma_ts(tm + o_col(s), tm + s_col(s) + Ly::P_OFF + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4),
                    idesc_pv, kk == 0 ? acc0 : 1u);
+            if constexpr (kLoP)
+              mma_ts(tm + o_col(s), tm + s_col(s) + Ly::P_OFF + 64 + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4),
+                     idesc_pv, 1u);
+          }
           first_pv[s] = false;
           if (rel_v[s]) mma_commit(&M.ring_empty[gv % NR]);
           pend_v[s] = -1;
@@ -886,7 +912,7 @@ static rola_status_t launch(const rola_shape_t* s, const uint16_t* q, const uint
       !rola_host::make_act_map(&mv, v, s, 128))
     return ROLA_ERR_CUDA;
   const size_t smem = Ly::misc_off + sizeof(Misc) + 1024;
-  auto kern = rola_attn_pair_kernel<R>;
+  auto kern = prm.out_lo ? rola_attn_pair_kernel<R, true> : rola_attn_pair_kernel<R, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ROLA_ERR_CUDA;
   const int nsm = rola_host::sm_count();
@@ -913,12 +939,13 @@ rola_status_t launch_pair_kernel(const rola_shape_t* s, const uint16_t* q, const
                                  const float* S_blk, const float* z_blk, const float* S_glb,
                                  const float* z_glb, const float* gate, uint16_t* out, int32_t* dev_err,
                                  const int32_t* kb_h, uint64_t wait_ns, float* lse, float* den,
-                                 cudaStream_t cs) {
+                                 uint16_t* out_lo, cudaStream_t cs) {
   pairk::Params prm{};
   prm.wait_ns = wait_ns;
   prm.kb_h = kb_h;
   prm.lse = lse;
   prm.den = den;
+  prm.out_lo = out_lo;
   prm.B = s->B;
   prm.H = s->H;
   prm.N = s->N;

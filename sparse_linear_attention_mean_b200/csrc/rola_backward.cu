@@ -103,6 +103,7 @@ struct Params {
   const float* S_glb;
   const float* z_glb;
   const uint16_t* out;
+  const uint16_t* out_lo;
   const uint16_t* dout;
   const float* lse;
   const float* den;
@@ -328,14 +329,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         lse2 = p.lse[ro] * 1.4426950408889634f;
         den = p.den[ro];
         c_row = lin ? g / den : 0.f;
-        const uint4* orow = reinterpret_cast<const uint4*>(p.out + ((b * (size_t)p.N + n) * p.H + h) * D);
-        const uint4* drow = reinterpret_cast<const uint4*>(p.dout + ((b * (size_t)p.N + n) * p.H + h) * D);
+        // D's first term dO . o from the output and its bf16 rounding residual
+        // (the rounding of o alone would cost D ~2^-9 of |dO| |o|)
+        const size_t ao = ((b * (size_t)p.N + n) * p.H + h) * D;
+        const uint4* orow = reinterpret_cast<const uint4*>(p.out + ao);
+        const uint4* lrow = reinterpret_cast<const uint4*>(p.out_lo + ao);
+        const uint4* drow = reinterpret_cast<const uint4*>(p.dout + ao);
 #pragma unroll 4
         for (int c = 0; c < D / 8; ++c) {
-          const uint4 o4 = __ldg(orow + c), d4 = __ldg(drow + c);
-          Dfull += bf16_lo(o4.x) * bf16_lo(d4.x) + bf16_hi(o4.x) * bf16_hi(d4.x) + bf16_lo(o4.y) * bf16_lo(d4.y) +
-                   bf16_hi(o4.y) * bf16_hi(d4.y) + bf16_lo(o4.z) * bf16_lo(d4.z) + bf16_hi(o4.z) * bf16_hi(d4.z) +
-                   bf16_lo(o4.w) * bf16_lo(d4.w) + bf16_hi(o4.w) * bf16_hi(d4.w);
+          const uint4 o4 = __ldg(orow + c), l4 = __ldg(lrow + c), d4 = __ldg(drow + c);
+          const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, lw[4] = {l4.x, l4.y, l4.z, l4.w};
+          const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            Dfull += (bf16_lo(ow[i]) + bf16_lo(lw[i])) * bf16_lo(dw[i]) +
+                     (bf16_hi(ow[i]) + bf16_hi(lw[i])) * bf16_hi(dw[i]);
         }
         coords(n, p.Hg, p.W, pt, py, px);
       }
@@ -579,8 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++ph_p;
         tc_fence_after();
         const uint32_t sK = smem_u32(smem + L::ring_off + (2 * st) * TILE);
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int kk = 0; kk < BN / 16; ++kk) {
           mma_ts(tm + kQ_dq, tm + kQ_S + kk * 8, desc_mnmaj(sK, BN, kk), id_pv, 1);
+          mma_ts(tm + kQ_dq, tm + kQ_dP + kk * 8, desc_mnmaj(sK, BN, kk), id_pv, 1);
+        }
         mma_commit(&M.empty[st]);
         const uint32_t my = ce[st]++;
         if (t + 1 < nk && !(ok = issue_s(t + 1))) break;
@@ -601,9 +611,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int blk = M.list[t];
         const int kvalid = min(BN, p.N - blk * BN);
+        // dS as bf16 hi (over the read S columns) + lo (over the read dP
+        // columns): dq sums dS K over the kept keys with cancellation, where
+        // the bf16 rounding of dS alone is ~2^-9 of sum |dS K|
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t sv[32], dv[32], pk[16];
+          uint32_t sv[32], dv[32], pk[16], pl[16];
           tmem_ld32(trow + kQ_S + c * 32, sv);
           tmem_ld32(trow + kQ_dP + c * 32, dv);
           tmem_wait_ld();
@@ -612,10 +625,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c0 = c * 32 + 2 * e;
             const float p0 = c0 < kvalid ? fast_exp2(__uint_as_float(sv[2 * e]) * p.scale_log2 - lse2) : 0.f;
             const float p1 = c0 + 1 < kvalid ? fast_exp2(__uint_as_float(sv[2 * e + 1]) * p.scale_log2 - lse2) : 0.f;
-            pk[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - Dv) * p.scale,
-                              p1 * (__uint_as_float(dv[2 * e + 1]) - Dv) * p.scale);
+            const float d0 = p0 * (__uint_as_float(dv[2 * e]) - Dv) * p.scale;
+            const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - Dv) * p.scale;
+            pk[e] = pack_bf16(d0, d1);
+            pl[e] = pack_bf16(d0 - bf16_lo(pk[e]), d1 - bf16_hi(pk[e]));
           }
           tmem_st16(trow + kQ_S + c * 16, pk);
+          tmem_st16(trow + kQ_dP + c * 16, pl);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -818,6 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < BM / 16; ++kk) {
           mma_ts(tm + kK_dV, tm + kK_S + kk * 8, desc_mnmaj(sOa, BM, kk), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
           mma_ts(tm + kK_dK, tm + kK_dP + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tm + kK_dK, tm + kK_S + 64 + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, 1u);
         }
         mma_commit(&M.empty[st]);
         const uint32_t my = ce[st]++;
@@ -847,7 +864,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++ph_s;
         if (!ok) continue;
         tc_fence_after();
-#pragma unroll 1
+        // P^T (bf16) over the read S^T columns [0, 64), dS^T hi over the read
+        // dP^T columns [0, 64), dS^T lo (held until every S^T column is read)
+        // over S^T columns [64, 128)
+        uint32_t dl[64];
+#pragma unroll
         for (int c = 0; c < BM / 32; ++c) {
           uint32_t sv[32], dv[32], pp[16], ds[16];
           tmem_ld32(trow + kK_S + c * 32, sv);
@@ -859,11 +880,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) * p.scale_log2 - M.lse2[st][q0]);
             const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) * p.scale_log2 - M.lse2[st][q0 + 1]);
             pp[e] = pack_bf16(p0, p1);
-            ds[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - M.Dr[st][q0]) * p.scale,
-                              p1 * (__uint_as_float(dv[2 * e + 1]) - M.Dr[st][q0 + 1]) * p.scale);
+            const float d0 = p0 * (__uint_as_float(dv[2 * e]) - M.Dr[st][q0]) * p.scale;
+            const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - M.Dr[st][q0 + 1]) * p.scale;
+            ds[e] = pack_bf16(d0, d1);
+            dl[c * 16 + e] = pack_bf16(d0 - bf16_lo(ds[e]), d1 - bf16_hi(ds[e]));
           }
           tmem_st16(trow + kK_S + c * 16, pp);
           tmem_st16(trow + kK_dP + c * 16, ds);
+          // S^T columns [64, 96) are read once chunk 2 is, [96, 128) with chunk 3
+          if (c == 2) tmem_st32_at<0>(trow + kK_S + 64, dl);
+          if (c == 3) tmem_st32_at<32>(trow + kK_S + 96, dl);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -1155,16 +1181,17 @@ extern "C" rola_status_t rola_attention_bwd(const rola_shape_t* s, const uint16_
                                             const uint16_t* v, const int32_t* idx, const uint16_t* P,
                                             const float* S_blk, const float* z_blk, const float* S_glb,
                                             const float* z_glb, const float* gate, const uint16_t* out,
-                                            const float* lse, const float* den, const uint16_t* dout,
+                                            const uint16_t* out_lo, const float* lse, const float* den,
+                                            const uint16_t* dout,
                                             uint16_t* dq, uint16_t* dk, uint16_t* dv, float* dP, float* dgate,
                                             void* ws, size_t ws_bytes, int32_t* dev_err, void* stream) {
   rola_status_t st = rola_internal::check_shape(s);
   if (st != ROLA_OK) return st;
-  if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out || !lse || !den ||
-      !dout || !dq || !dk || !dv || !dP || !dgate)
+  if (!q || !k || !v || !idx || !P || !S_blk || !z_blk || !S_glb || !z_glb || !gate || !out || !out_lo || !lse ||
+      !den || !dout || !dq || !dk || !dv || !dP || !dgate)
     return ROLA_ERR_INVALID_ARG;
   if (!bwd::bwd_supports(s)) return ROLA_ERR_UNSUPPORTED;
-  const void* a16[] = {q, k, v, out, dout, dq, dk, dv};
+  const void* a16[] = {q, k, v, out, out_lo, dout, dq, dk, dv};
   for (const void* ptr : a16)
     if (!rola_host::aligned(ptr, 16)) return ROLA_ERR_ALIGNMENT;
   const void* a4[] = {idx, S_blk, z_blk, S_glb, z_glb, gate, lse, den, dP, dgate};
@@ -1193,6 +1220,7 @@ extern "C" rola_status_t rola_attention_bwd(const rola_shape_t* s, const uint16_
   prm.S_glb = S_glb;
   prm.z_glb = z_glb;
   prm.out = out;
+  prm.out_lo = out_lo;
   prm.dout = dout;
   prm.lse = lse;
   prm.den = den;
