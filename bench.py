@@ -344,6 +344,7 @@ def run_gpu(args) -> int:
             line["per_config"] = {str(i): config_report(i, stream, peaks, flush, 10, 50)
                                   for i in (0, 1, 2, 3)}
             line["per_config"]["4"] = block_report(stream, peaks, flush, 3, 10)
+            line["training"] = backward_report(args.workload, stream, peaks, flush, 3, 10)
         if not args.no_cpu_baseline and world == 1:
             # the host-core oracle is timed at one GPU only (the multi-GPU
             # lines keep the other ranks waiting as little as possible)
@@ -408,6 +409,22 @@ def _timed_reps(fn, stream, flush, warmup: int, reps: int, n_events: int = 2):
     return [[ev[i].elapsed_time(ev[i + 1]) for i in range(n_events - 1)] for ev in evs]
 
 
+def unit_overlap(idx: np.ndarray) -> dict:
+    """Mean size of the union and of the intersection of the kept lists of the
+    two query blocks (2p, 2p + 1) that the attention kernel pairs in a unit
+    (padding entries -1 ignored)."""
+    B, H, nb, _ = idx.shape
+    uni, inter = [], []
+    for b in range(B):
+        for h in range(H):
+            for p in range(0, nb, 2):
+                a = set(int(x) for x in idx[b, h, p] if x >= 0)
+                c = set(int(x) for x in idx[b, h, p + 1] if x >= 0) if p + 1 < nb else set()
+                uni.append(len(a | c))
+                inter.append(len(a & c))
+    return {"units": len(uni), "union_mean": float(np.mean(uni)), "shared_mean": float(np.mean(inter))}
+
+
 def config_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
     """One attention workload through the layer entry point: ms per layer and
     per stage (p50 / p95), effective TFLOP/s of the layer and of the attention
@@ -465,7 +482,63 @@ def config_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) 
                     bad += 1
     rep["mask"] = {"rows": int(w.B * w.H * w.n_blocks), "mismatch_outside_near_ties": bad,
                    "near_tie_rows": n_tie_rows, "differing_near_tie_rows": ties}
+    rep["unit_lists"] = unit_overlap(got)
     del q, k, v, out, layer
+    torch.cuda.empty_cache()
+    return rep
+
+
+def backward_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
+    """Training on one attention workload: the training forward (which also
+    saves the output residual, log-sum-exp and linear denominator) and the
+    backward (transposed mask, query-major and key-major tcgen05 passes,
+    fixed-order reductions), each timed alone with an L2 flush before every
+    rep.  TFLOP/s count the kept pairs' contractions as the usual dense
+    accounting does: 2 per pair forward, 5 backward (S recomputed, dP, dQ,
+    dK, dV); the two-pass backward executes 7 (S and dP in both passes)."""
+    import ctypes
+
+    import torch
+    from sparse_linear_attention_mean_b200 import binding as rb
+    from sparse_linear_attention_mean_b200 import synth
+    w = synth.WORKLOADS[wid]
+    shape = rb.Shape.of(w)
+    inp = synth.make_inputs(w)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
+    q, k, v, P = dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["P"])
+    gate = torch.from_numpy(inp["gate"]).cuda()
+    dout = dev(synth.make_normal_bf16((w.B, w.N, w.H, w.d), seed=w.seed + 50, stream=7))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx = rb.select_blocks(shape, q, k, stream=stream)
+    states = rb.block_states(shape, k, v, P, stream=stream)
+    fwd = rb.attention_fwd_train(shape, q, k, v, idx, P, states, gate, dev_err=err, stream=stream)
+    grads = rb.attention_bwd(shape, q, k, v, idx, P, states, gate, *fwd, dout, dev_err=err, stream=stream)
+    ws = torch.empty(rb.lib().rola_attention_bwd_workspace_bytes(ctypes.byref(shape.c())),
+                     dtype=torch.uint8, device="cuda")
+
+    def f_fwd(ev):
+        ev[0].record(stream)
+        rb.attention_fwd_train(shape, q, k, v, idx, P, states, gate, dev_err=err, stream=stream)
+        ev[1].record(stream)
+
+    def f_bwd(ev):
+        ev[0].record(stream)
+        rb.attention_bwd(shape, q, k, v, idx, P, states, gate, *fwd, dout, dev_err=err, stream=stream,
+                         workspace=ws, grads=grads)
+        ev[1].record(stream)
+
+    t_f = [x[0] for x in _timed_reps(f_fwd, stream, flush, warmup, reps)]
+    t_b = [x[0] for x in _timed_reps(f_bwd, stream, flush, warmup, reps)]
+    assert int(err.item()) == 0
+    flop_fwd = w.sparse_flops()
+    rep = {"workload": w.name, "reps": reps, "warmup": warmup, "l2": "256 MB flush before each rep",
+           "train_forward_ms_p50": _pct(t_f, 50), "train_forward_ms_p95": _pct(t_f, 95),
+           "backward_ms_p50": _pct(t_b, 50), "backward_ms_p95": _pct(t_b, 95)}
+    rep["train_forward_tflops"] = flop_fwd / (rep["train_forward_ms_p50"] * 1e-3) / 1e12
+    rep["backward_tflops"] = 2.5 * flop_fwd / (rep["backward_ms_p50"] * 1e-3) / 1e12
+    rep["backward_tflops_executed"] = 3.5 * flop_fwd / (rep["backward_ms_p50"] * 1e-3) / 1e12
+    rep["backward_frac_of_bf16_peak"] = rep["backward_tflops"] / peaks["bf16_tflops"]
+    del q, k, v, P, dout, fwd, grads, ws, states, idx
     torch.cuda.empty_cache()
     return rep
 
@@ -506,6 +579,8 @@ def block_report(stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
     def gemm(wq, ws, dst):
         assert lib.fp8_gemm_w8a8(M, D, D, P_(xq), P_(xs), P_(wq), P_(ws), P_(dst), P_(err), cs) == 0
 
+    idx = torch.empty((w.B, w.H, w.n_blocks, w.k_b), dtype=torch.int32, device="cuda")
+
     def step(ev):
         ev[0].record(stream)
         quant(x)
@@ -513,7 +588,8 @@ def block_report(stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
             gemm(*wts[nm], qkv[nm])
         ev[1].record(stream)
         layer(qkv["Wq"].view(w.B, w.N, w.H, w.d), qkv["Wk"].view(w.B, w.N, w.H, w.d),
-              qkv["Wv"].view(w.B, w.N, w.H, w.d), P, gate, out=o.view(w.B, w.N, w.H, w.d), stream=stream)
+              qkv["Wv"].view(w.B, w.N, w.H, w.d), P, gate, out=o.view(w.B, w.N, w.H, w.d), idx_out=idx,
+              stream=stream)
         ev[2].record(stream)
         quant(o)
         gemm(*wts["Wo"], y)
@@ -536,7 +612,8 @@ def block_report(stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
     rep["qkv_frac_of_fp8_peak"] = rep["qkv_tflops"] / fp8_peak
     rep["out_tflops"] = gflop / (rep["quant+out_gemm_ms_p50"] * 1e-3) / 1e12
     rep["out_frac_of_fp8_peak"] = rep["out_tflops"] / fp8_peak
-    del qkv, o, layer
+    rep["unit_lists"] = unit_overlap(idx.cpu().numpy())
+    del qkv, o, layer, idx
     torch.cuda.empty_cache()
     # the block's FFN
     ffw = synth.make_ffn_weights(w)

@@ -276,16 +276,24 @@ def attention_fwd_train(shape: Shape, q, k, v, idx, P, states, gate, *, dev_err=
 
 
 def attention_bwd(shape: Shape, q, k, v, idx, P, states, gate, out, out_lo, lse, den, dout, *, dev_err=None,
-                  stream=None, workspace=None):
+                  stream=None, workspace=None, grads=None):
     """Gradients (dq, dk, dv bf16 [B, N, H, d], dP float [H, d, r], dgate
-    float [H]) of sum(dout * out) for the forward of attention_fwd_train."""
+    float [H]) of sum(dout * out) for the forward of attention_fwd_train.
+    `grads`, if given, is that tuple preallocated (every element is written)."""
     act = (shape.B, shape.N, shape.H, shape.d)
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (out_lo, "out_lo"), (dout, "dout")):
         _need(t, torch.bfloat16, act, nm)
     S_blk, z_blk, S_glb, z_glb = states
-    dq, dk, dv = (torch.zeros(act, dtype=torch.bfloat16, device=q.device) for _ in range(3))
-    dP = torch.empty((shape.H, shape.d, shape.r), dtype=torch.float32, device=q.device)
-    dgate = torch.empty((shape.H,), dtype=torch.float32, device=q.device)
+    if grads is None:
+        dq, dk, dv = (torch.empty(act, dtype=torch.bfloat16, device=q.device) for _ in range(3))
+        dP = torch.empty((shape.H, shape.d, shape.r), dtype=torch.float32, device=q.device)
+        dgate = torch.empty((shape.H,), dtype=torch.float32, device=q.device)
+    else:
+        dq, dk, dv, dP, dgate = grads
+        for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+            _need(t, torch.bfloat16, act, nm)
+        _need(dP, torch.float32, (shape.H, shape.d, shape.r), "dP")
+        _need(dgate, torch.float32, (shape.H,), "dgate")
     c = shape.c()
     nbytes = lib().rola_attention_bwd_workspace_bytes(ctypes.byref(c))
     if nbytes == 0:
