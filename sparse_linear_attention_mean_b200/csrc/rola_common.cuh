@@ -104,6 +104,8 @@ ROLA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   uint32_t spins = 0;
+  // try_wait itself suspends the thread for a while; no sleep between
+  // attempts (a sleeping waiter answers a completed phase later)
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (++spins > 64) {
@@ -112,7 +114,6 @@ ROLA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
         *abort = 1;
         return false;
       }
-      __nanosleep(64);
     }
   }
 }
