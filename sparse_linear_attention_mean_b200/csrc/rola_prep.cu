@@ -8,9 +8,10 @@
 // (per-block states S_j = rho^T V, z_j = sum psi, rho = R(t, y, x) phi(K P_h)).
 //
 // Persistent CTAs (256 threads, two per SM) walk (batch, head, block) items.
-// Thread 0 TMA-loads the item's k and v tiles (128-byte swizzle) while every
-// thread loads its share of the q tile straight into registers; the other
-// CTA on the SM computes meanwhile.  Per item:
+// Thread 0 TMA-loads an item's k and v tiles (128-byte swizzle) and every
+// thread loads its share of its q tile straight into registers while the
+// previous item is still being computed: k and q once the previous item's
+// pooling has consumed them, v once its state product has.  Per item:
 //   * K P_h with mma.sync (first: it needs only the k tile, so the q loads
 //     have this long to land);
 //   * block sums of q and k over the valid tokens in float64 (exact for bf16;
@@ -46,7 +47,7 @@ struct Layout {
 };
 
 struct Misc {
-  uint64_t full;
+  uint64_t full_k, full_v;
   int abort;
   int cur_h;
   float zpart[8][32];
@@ -124,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int my_items = max(0, min(per_cta, p.items - first_item));
 
   if (tid == 0) {
-    mbar_init(&M.full, 1);
+    mbar_init(&M.full_k, 1);
+    mbar_init(&M.full_v, 1);
     M.abort = 0;
     M.cur_h = -1;
     fence_barrier_init();
@@ -146,28 +148,52 @@ __global__ void __launch_bounds__(kThreads, 2)
     h = (id / p.nb) % p.H;
     b = id / (p.nb * p.H);
   };
-  auto issue = [&](int it) {
+  // The k and v tiles of an item go to their buffers as soon as the previous
+  // item is done with them: k after its pooling, v after its state product,
+  // so that each copy overlaps the rest of the previous item.
+  auto issue_k = [&](int it) {
     int b, h, blk;
     decode(it, b, h, blk);
-    mbar_expect_tx(&M.full, 2 * TILE);
-    for (int ka = 0; ka < 2; ++ka) {
-      tma_load_4d(smem + ka * (BS * 128), &tmK, &M.full, ka * 64, h, blk * BS, b);
-      tma_load_4d(smem + TILE + ka * (BS * 128), &tmV, &M.full, ka * 64, h, blk * BS, b);
+    mbar_expect_tx(&M.full_k, TILE);
+    for (int ka = 0; ka < 2; ++ka) tma_load_4d(smem + ka * (BS * 128), &tmK, &M.full_k, ka * 64, h, blk * BS, b);
+  };
+  auto issue_v = [&](int it) {
+    int b, h, blk;
+    decode(it, b, h, blk);
+    mbar_expect_tx(&M.full_v, TILE);
+    for (int ka = 0; ka < 2; ++ka)
+      tma_load_4d(smem + TILE + ka * (BS * 128), &tmV, &M.full_v, ka * 64, h, blk * BS, b);
+  };
+  // pooling: thread = (row group rg of rows rg + 16 i, 8-channel chunk c8)
+  const int rg = tid >> 4, c8 = tid & 15;
+  double* part = reinterpret_cast<double*>(smem + Ly::rho_off);  // [8][2][D]
+  // this thread's share of an item's q tile, straight into registers (it
+  // is loaded for the next item as soon as this item's pooling is done)
+  uint4 qv[8];
+  auto load_q = [&](int it) {
+    int b, h, blk;
+    decode(it, b, h, blk);
+    const int tok0 = blk * BS, valid = min(BS, p.N - tok0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = rg + 16 * i;
+      qv[i] = row < valid ? __ldg(reinterpret_cast<const uint4*>(
+                                p.q + (((size_t)b * p.N + tok0 + row) * p.H + h) * D + c8 * 8))
+                          : make_uint4(0, 0, 0, 0);
     }
   };
   if (tid == 0 && my_items > 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    issue_k(0);
+    issue_v(0);
   }
-  // pooling: thread = (row group rg of rows rg + 16 i, 8-channel chunk c8)
-  const int rg = tid >> 4, c8 = tid & 15;
-  double* part = reinterpret_cast<double*>(smem + Ly::rho_off);  // [8][2][D]
+  if (p.do_pool && my_items > 0) load_q(0);
+  int k_issued = my_items > 0 ? 1 : 0, v_issued = k_issued;  // copies issued (thread 0's count)
 
   bool ok = true;
   int it = 0;
   for (; ok && it < my_items; ++it) {
-    // the stage was released by the __syncthreads closing the last item
-    if (tid == 0) issue(it);
     int b, h, blk;
     decode(it, b, h, blk);
     const size_t bh = (size_t)b * p.H + h;
@@ -175,16 +201,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int valid = min(BS, p.N - tok0);
     uint8_t* sk = smem;
     uint8_t* sv = sk + TILE;
-    uint4 qv[8];
-    if (p.do_pool) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int row = rg + 16 * i;
-        qv[i] = row < valid ? __ldg(reinterpret_cast<const uint4*>(
-                                  p.q + (((size_t)b * p.N + tok0 + row) * p.H + h) * D + c8 * 8))
-                            : make_uint4(0, 0, 0, 0);
-      }
-    }
     // P_h (rows d, padded) when the head changes
     if (h != M.cur_h) {
       for (int e = tid; e < D * (R / 8); e += kThreads) {
@@ -195,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncthreads();
       if (tid == 0) M.cur_h = h;
     }
-    if (!(ok = mbar_wait(&M.full, it & 1, abort))) break;
+    if (!(ok = __syncthreads_and(mbar_wait(&M.full_k, it & 1, abort)))) break;
 
     // ---- kt = K P_h : warp w owns token rows [16w, 16w + 16)
     constexpr int NT = R / 8;
@@ -255,7 +271,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
-    __syncthreads();  // pooling partials complete
+    __syncthreads();  // pooling partials complete; k and this thread's q are consumed
+    if (it + 1 < my_items) {
+      if (tid == 0) {
+        issue_k(it + 1);
+        ++k_issued;
+      }
+      if (p.do_pool) load_q(it + 1);
+    }
     if (p.do_pool) {
       const int tile = tid >> 7, c = tid & 127;
       double acc2 = 0.0;
@@ -317,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     // ---- S_j^T pieces: C[r, d] = rho^T V, warp w owns d columns [16w, 16w + 16)
+    if (!(ok = __syncthreads_and(mbar_wait(&M.full_v, it & 1, abort)))) break;
     {
       constexpr int MT = R / 16;
       float c2[MT][2][4];
@@ -355,12 +379,18 @@ __global__ void __launch_bounds__(kThreads, 2)
               make_float2(c2[mi][nj][2], c2[mi][nj][3]);
         }
     }
-    __syncthreads();  // stage st is free for item it + 2
+    __syncthreads();  // v is consumed
+    if (tid == 0 && it + 1 < my_items) {
+      issue_v(it + 1);
+      ++v_issued;
+    }
   }
-  // drain: if we stopped early, let the copy in flight land before exiting
-  if (tid == 0 && it < my_items) {
+  // drain: if we stopped early, let the copies in flight land before exiting
+  // (copy i completes phase i of its barrier; items < it were waited for)
+  if (tid == 0) {
     int no_abort = 0;
-    mbar_wait(&M.full, it & 1, &no_abort);
+    for (int i = it; i < k_issued; ++i) mbar_wait(&M.full_k, i & 1, &no_abort);
+    for (int i = it; i < v_issued; ++i) mbar_wait(&M.full_v, i & 1, &no_abort);
   }
   if (tid == 0 && M.abort && p.dev_err) atomicOr(p.dev_err, ROLA_DEVERR_TIMEOUT);
 }
