@@ -711,6 +711,8 @@ def main() -> int:
     ap.add_argument("--fp8-only", action="store_true",
                     help="time only the FP8 projection (x [rows, 5120] -> [rows, 5120]); profiling captures")
     ap.add_argument("--fp8-rows", type=int, default=75600, help="rows of x for --fp8-only")
+    ap.add_argument("--training-only", action="store_true",
+                    help="time only the training forward and the backward of --workload; profiling captures")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (per-head work unchanged; for profiling captures)")
     ap.add_argument("--workload", type=int, default=WORKLOAD_ID,
@@ -721,6 +723,12 @@ def main() -> int:
     if args.fp8_only:
         import torch
         print(json.dumps({"fp8_projection": fp8_projection(args.fp8_rows, 5120, torch.cuda.current_stream())}))
+        return 0
+    if args.training_only:
+        import torch
+        stream = torch.cuda.current_stream()
+        print(json.dumps({"training": backward_report(args.workload, stream, measured_peaks(), L2Flush(),
+                                                      args.warmup, args.steps)}))
         return 0
     return run_gpu(args)
 
