@@ -85,10 +85,7 @@ ROLA_DEV void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
 }
 
 // 3-D rotary pair of a token (t, y, x); pair pr turns by pos(axis) * freq.
-ROLA_DEV void rope_cs(const RopeTable& rt, int pr, int pt, int py, int px, float& c, float& s) {
-  const int ax = rt.axis[pr];
-  rope_sincos(ax == 0 ? pt : (ax == 1 ? py : px), rt.freq[pr], &s, &c);
-}
+constexpr int kTabCap = 1024;  // cos/sin entries of the rotary table in shared memory
 
 struct Params {
   int B, H, N, nb, kb, T, Hg, W;
@@ -122,7 +119,30 @@ struct Params {
   int chunks_q, chunks_k;
   int32_t* dev_err;
   RopeTable rope;
+  // rotary table: entry of pair pr at position pos = tab_base[pr] + pos * tab_stride[pr];
+  // pair pr fills entries [tab_first[pr], tab_first[pr + 1]) of the fill order
+  int tab_base[16], tab_stride[16], tab_first[17];
+  int tab_entries;
 };
+
+// (cos, sin) of rotation pair pr at the row's grid position, from the table
+ROLA_DEV void rope_cs(const Params& p, const float2* tab, int pr, int pt, int py, int px, float& c, float& s) {
+  const int ax = p.rope.axis[pr];
+  const float2 v = tab[p.tab_base[pr] + (ax == 0 ? pt : (ax == 1 ? py : px)) * p.tab_stride[pr]];
+  c = v.x;
+  s = v.y;
+}
+// The table, once per CTA: the same rope_sincos values the forward's table holds.
+ROLA_DEV void fill_rope_table(const Params& p, float2* tab, int R, int nthreads) {
+  for (int e = (int)threadIdx.x; e < p.tab_entries; e += nthreads) {
+    int pr = 0;
+    while (pr + 1 < R / 2 && e >= p.tab_first[pr + 1]) ++pr;
+    const int pos = e - p.tab_first[pr];
+    float sn, cs;
+    rope_sincos(pos, p.rope.freq[pr], &sn, &cs);
+    tab[p.tab_base[pr] + pos * p.tab_stride[pr]] = make_float2(cs, sn);
+  }
+}
 
 // ================================================================ transposed mask
 // One CTA per (b, h): bits[j][w] bit (a & 31) of word a >> 5 is set when query
@@ -233,6 +253,7 @@ struct QMisc {
   float red[4][32];
   float lse2[BM];
   float Dr[BM];
+  float2 tab[kTabCap];
 };
 
 // TMEM columns of the query-major kernel
@@ -275,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&M.tmem, 512);
     tmem_relinquish();
   }
+  fill_rope_table(p, M.tab, R, kThreads);
   // P_h operands of this head: P_h^T (SW128 K-major, N = r rows, K = d) and
   // P_h (core K-major, N = d rows, K = r); P_h is bf16, so no lo part
   for (int e = tid; e < D * R; e += kThreads) {
@@ -411,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int pr = 0; pr < R / 2; ++pr) {
         float cs, sn;
-        rope_cs(p.rope, pr, pt, py, px, cs, sn);
+        rope_cs(p, M.tab, pr, pt, py, px, cs, sn);
         const float r0 = psi[2 * pr] * cs - psi[2 * pr + 1] * sn;
         const float r1 = psi[2 * pr] * sn + psi[2 * pr + 1] * cs;
         uint16_t h0, l0, h1, l1;
@@ -487,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int pr = 0; pr < R / 2; ++pr) {
         float cs, sn;
-        rope_cs(p.rope, pr, pt, py, px, cs, sn);
+        rope_cs(p, M.tab, pr, pt, py, px, cs, sn);
         const float d0 = c_row * __uint_as_float(w[2 * pr]), d1 = c_row * __uint_as_float(w[2 * pr + 1]);
         // R^T of the pair rotation: (d0 cs + d1 sn, -d0 sn + d1 cs)
         const float p0 = dden * M.zU[2 * pr] + d0 * cs + d1 * sn;
@@ -713,6 +735,7 @@ struct KMisc {
   float zb[32];
   float lse2[2][BM];
   float Dr[2][BM];
+  float2 tab[kTabCap];
 };
 
 // TMEM columns of the key-major kernel
@@ -752,6 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&M.tmem, 512);
     tmem_relinquish();
   }
+  fill_rope_table(p, M.tab, R, kThreads);
   for (int e = tid; e < D * R; e += kThreads) {
     const int c = e / R, rr = e % R;
     const uint16_t w = p.P[((size_t)h * D + c) * R + rr];
@@ -949,7 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int pr = 0; pr < R / 2; ++pr) {
         float cs, sn;
-        rope_cs(p.rope, pr, kpt, kpy, kpx, cs, sn);
+        rope_cs(p, M.tab, pr, kpt, kpy, kpx, cs, sn);
         const float r0 = kvalid ? psik[2 * pr] * cs - psik[2 * pr + 1] * sn : 0.f;
         const float r1 = kvalid ? psik[2 * pr] * sn + psik[2 * pr + 1] * cs : 0.f;
         uint16_t h0, l0, h1, l1;
@@ -993,7 +1017,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int pr = 0; pr < R / 2; ++pr) {
         float cs, sn;
-        rope_cs(p.rope, pr, kpt, kpy, kpx, cs, sn);
+        rope_cs(p, M.tab, pr, kpt, kpy, kpx, cs, sn);
         const float d0 = __uint_as_float(w[2 * pr]), d1 = __uint_as_float(w[2 * pr + 1]);
         const float p0 = M.zb[2 * pr] + d0 * cs + d1 * sn;
         const float p1 = M.zb[2 * pr + 1] - d0 * sn + d1 * cs;
@@ -1240,6 +1264,15 @@ extern "C" rola_status_t rola_attention_bwd(const rola_shape_t* s, const uint16_
   prm.chunks_k = W.ck;
   prm.dev_err = dev_err;
   rola_host::rope_frequencies(s->r, s->rope_base, prm.rope.freq, prm.rope.axis);
+  rola_host::RopeTabLayout tl;
+  rola_host::rope_table_layout(s, prm.rope.axis, &tl);
+  if (tl.entries > bwd::kTabCap) return ROLA_ERR_UNSUPPORTED;
+  for (int i = 0; i < 16; ++i) {
+    prm.tab_base[i] = tl.base[i];
+    prm.tab_stride[i] = tl.stride[i];
+  }
+  for (int i = 0; i < 17; ++i) prm.tab_first[i] = tl.first[i];
+  prm.tab_entries = tl.entries;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   st = s->r == 32 ? bwd::launch_bwd<32>(s, q, k, v, dout, prm, W, base, cs)
                   : bwd::launch_bwd<16>(s, q, k, v, dout, prm, W, base, cs);
