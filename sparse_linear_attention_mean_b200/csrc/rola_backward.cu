@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         u[i] = valid ? __uint_as_float(v[i]) : 0.f;
-        psi[i] = phi(u[i]);
+        psi[i] = phi_fast(u[i]);
       }
       // rho (core K-major A) and (c rho)^T (SW128 K-major B over the rows)
 #pragma unroll
@@ -968,7 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < R; ++i) {
         uk[i] = kvalid ? __uint_as_float(v[i]) : 0.f;
-        psik[i] = phi(uk[i]);
+        psik[i] = phi_fast(uk[i]);
       }
 #pragma unroll
       for (int pr = 0; pr < R / 2; ++pr) {
