@@ -346,27 +346,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     float lse2 = INFINITY, c_row = 0.f, den = 1.f, Dfull = 0.f;
     int pt = 0, py = 0, px = 0;
     if (tid < kCompute) {
+      // D's first term dO . o, from the output and its bf16 rounding residual
+      // (the rounding of o alone would cost D ~2^-9 of |dO| |o|).  A warp
+      // reads its 32 rows two at a time, 16 lanes x 16 bytes per row of each
+      // of out, out_lo and dout (coalesced), and sums each row over its 16
+      // lanes; row i's sum lands in M.Dr[i] for its owner thread.
+      {
+        const int half = lane >> 4, l16 = lane & 15;
+#pragma unroll 4
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const int r = warp * 32 + 2 * i2 + half, nr = a * BM + r;
+          float part = 0.f;
+          if (nr < p.N) {
+            const size_t ao = ((b * (size_t)p.N + nr) * p.H + h) * D + l16 * 8;
+            const uint4 o4 = __ldg(reinterpret_cast<const uint4*>(p.out + ao));
+            const uint4 l4 = __ldg(reinterpret_cast<const uint4*>(p.out_lo + ao));
+            const uint4 d4 = __ldg(reinterpret_cast<const uint4*>(p.dout + ao));
+            const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, lw[4] = {l4.x, l4.y, l4.z, l4.w};
+            const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              part += (bf16_lo(ow[i]) + bf16_lo(lw[i])) * bf16_lo(dw[i]) +
+                      (bf16_hi(ow[i]) + bf16_hi(lw[i])) * bf16_hi(dw[i]);
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          if (l16 == 0) M.Dr[r] = part;
+        }
+        __syncwarp();
+      }
       if (valid) {
         const size_t ro = bh * p.N + n;
         lse2 = p.lse[ro] * 1.4426950408889634f;
         den = p.den[ro];
         c_row = lin ? g / den : 0.f;
-        // D's first term dO . o from the output and its bf16 rounding residual
-        // (the rounding of o alone would cost D ~2^-9 of |dO| |o|)
-        const size_t ao = ((b * (size_t)p.N + n) * p.H + h) * D;
-        const uint4* orow = reinterpret_cast<const uint4*>(p.out + ao);
-        const uint4* lrow = reinterpret_cast<const uint4*>(p.out_lo + ao);
-        const uint4* drow = reinterpret_cast<const uint4*>(p.dout + ao);
-#pragma unroll 4
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 o4 = __ldg(orow + c), l4 = __ldg(lrow + c), d4 = __ldg(drow + c);
-          const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, lw[4] = {l4.x, l4.y, l4.z, l4.w};
-          const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            Dfull += (bf16_lo(ow[i]) + bf16_lo(lw[i])) * bf16_lo(dw[i]) +
-                     (bf16_hi(ow[i]) + bf16_hi(lw[i])) * bf16_hi(dw[i]);
-        }
+        Dfull = M.Dr[tid];
         coords(n, p.Hg, p.W, pt, py, px);
       }
       // S_U column d = tid: S - sum over the kept blocks (fp32, as the forward)
@@ -375,7 +389,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int r = 0; r < R; ++r) su[r] = Sg[r * D + tid];
       float zu = tid < R ? p.z_glb[bh * R + tid] : 0.f;
-      for (int e = 0; e < nk; ++e) {
+      // four blocks' loads in flight per round trip; the subtractions keep
+      // the kept list's order
+      int e = 0;
+      for (; e + 4 <= nk; e += 4) {
+        float t[4][R];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float* Sb = p.S_blk + (bh * p.nb + M.list[e + i]) * R * D;
+#pragma unroll
+          for (int r = 0; r < R; ++r) t[i][r] = __ldg(Sb + r * D + tid);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int r = 0; r < R; ++r) su[r] -= t[i][r];
+        if (tid < R)
+          for (int i = 0; i < 4; ++i) zu -= p.z_blk[(bh * p.nb + M.list[e + i]) * R + tid];
+      }
+      for (; e < nk; ++e) {
         const size_t st = bh * p.nb + M.list[e];
         const float* Sb = p.S_blk + st * R * D;
 #pragma unroll
@@ -932,7 +964,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int r = 0; r < R; ++r) sb[r] = p.dSU_tot[bh * R * D + r * D + tid];
       float zb = tid < R ? p.dzU_tot[bh * R + tid] : 0.f;
-      for (int t = 0; t < nkeep; ++t) {
+      // four keepers' loads in flight per round trip; the subtractions keep
+      // the keepers' order
+      int t = 0;
+      for (; t + 4 <= nkeep; t += 4) {
+        float v4[4][R];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float* src = p.dSU + (bh * p.nb + M.keep[t + i]) * R * D;
+#pragma unroll
+          for (int r = 0; r < R; ++r) v4[i][r] = __ldcg(src + r * D + tid);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int r = 0; r < R; ++r) sb[r] -= v4[i][r];
+        if (tid < R)
+          for (int i = 0; i < 4; ++i) zb -= p.dzU[(bh * p.nb + M.keep[t + i]) * R + tid];
+      }
+      for (; t < nkeep; ++t) {
         const size_t st = bh * p.nb + M.keep[t];
 #pragma unroll
         for (int r = 0; r < R; ++r) sb[r] -= p.dSU[st * R * D + r * D + tid];
