@@ -124,10 +124,10 @@ def test_backward_dense_limit_every_block_kept():
     assert torch.all(dP == 0) and torch.all(dg == 0)
 
 
-@pytest.mark.parametrize("cfg,heads", [(1, [0, 11]), (3, [0])])
+@pytest.mark.parametrize("cfg,heads", [(1, [0, 11]), (2, [39]), (3, [0])])
 def test_backward_workloads(cfg, heads):
-    """Wan2.1-1.3B 480P (all rows of two heads) and 14B 720P (all rows of
-    head 0), at the nominal gate."""
+    """Wan2.1-1.3B 480P (all rows of two heads), 14B 480P (all rows of the
+    last head) and 14B 720P (all rows of head 0), at the nominal gate."""
     w = synth.WORKLOADS[cfg]
     inp = synth.make_inputs(w)
     idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
