@@ -242,7 +242,7 @@ struct QLayout {
 };
 
 struct QMisc {
-  uint64_t load, mma, s_ready, p_ready, full[2], empty[2];
+  uint64_t load, mma, s_ready, p_ready, full[2], empty[2], d_ready;
   uint32_t tmem;
   int abort;
   int err;
@@ -258,6 +258,7 @@ struct QMisc {
 
 // TMEM columns of the query-major kernel
 constexpr uint32_t kQ_dq = 0, kQ_S = 128, kQ_dP = 256, kQ_uq = 384, kQ_ds = 416, kQ_dsu = 448, kQ_dph = 480;
+constexpr uint32_t kQ_S2 = 384;  // the sparse loop's second S buffer (over the linear phase's columns)
 
 // ================================================================ query-major pass
 template <int R>
@@ -288,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&M.full[i], 1);
       mbar_init(&M.empty[i], 1);
     }
+    mbar_init(&M.d_ready, 1);
     M.abort = 0;
     M.err = 0;
     fence_barrier_init();
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const float g = p.gate[h];
   // phase counters of the barriers; ce counts the commits to empty[] (a
   // stage's commits outnumber the waits on it, so its parity follows the commits)
-  uint32_t ph_load = 0, ph_mma = 0, ph_s = 0, ph_p = 0, ph_full[2] = {0, 0}, ce[2] = {0, 0};
+  uint32_t ph_load = 0, ph_mma = 0, ph_s = 0, ph_p = 0, ph_full[2] = {0, 0}, ce[2] = {0, 0}, ph_d = 0;
   float dph[R];  // thread t (< 128) accumulates row t (= d index) of this CTA's P_h partial
 #pragma unroll
   for (int i = 0; i < R; ++i) dph[i] = 0.f;
@@ -619,35 +621,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                       blk * BN, b);
         }
       };
-      auto issue_s = [&](int t) -> bool {
+      // S of pair t goes to one of two buffers (columns 128 and 384; the
+      // latter hold the linear phase's operands, done by now), dP to one
+      auto sbuf = [](int t) -> uint32_t { return (t & 1) ? kQ_S2 : kQ_S; };
+      auto issue_S = [&](int t) -> bool {
         const int st = t & 1;
         if (!mbar_wait(&M.full[st], ph_full[st] & 1, abort)) return false;
         ++ph_full[st];
         tc_fence_after();
         const uint32_t sK = smem_u32(smem + L::ring_off + (2 * st) * TILE);
-        const uint32_t sV = sK + TILE;
-        for (int kk = 0; kk < D / 16; ++kk) {
-          mma_ss(tm + kQ_S, desc_kmaj(sQ, BM, kk), desc_kmaj(sK, BN, kk), id_dd, kk > 0);
-          mma_ss(tm + kQ_dP, desc_kmaj(sO, BM, kk), desc_kmaj(sV, BN, kk), id_dd, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tm + sbuf(t), desc_kmaj(sQ, BM, kk), desc_kmaj(sK, BN, kk), id_dd, kk > 0);
         mma_commit(&M.s_ready);
         return true;
       };
+      auto issue_dP = [&](int t) {
+        const uint32_t sV = smem_u32(smem + L::ring_off + (2 * (t & 1) + 1) * TILE);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tm + kQ_dP, desc_kmaj(sO, BM, kk), desc_kmaj(sV, BN, kk), id_dd, kk > 0);
+        mma_commit(&M.d_ready);
+      };
       for (int t = 0; t < min(nk, 2); ++t) load_kv(t);
-      if (nk > 0) ok = issue_s(0);
+      if (nk > 0 && (ok = issue_S(0))) issue_dP(0);
+      // per pair t: S(t + 1) first (the next pair's exponentials need only
+      // it), then dq += dS(t) K(t), then dP(t + 1) (it overwrites the dP
+      // columns, which hold dS(t)'s lo part until that MMA has read them)
       for (int t = 0; ok && t < nk; ++t) {
         const int st = t & 1;
         if (!(ok = mbar_wait(&M.p_ready, ph_p & 1, abort))) break;
         ++ph_p;
         tc_fence_after();
+        if (t + 1 < nk && !(ok = issue_S(t + 1))) break;
         const uint32_t sK = smem_u32(smem + L::ring_off + (2 * st) * TILE);
         for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tm + kQ_dq, tm + kQ_S + kk * 8, desc_mnmaj(sK, BN, kk), id_pv, 1);
+          mma_ts(tm + kQ_dq, tm + sbuf(t) + kk * 8, desc_mnmaj(sK, BN, kk), id_pv, 1);
           mma_ts(tm + kQ_dq, tm + kQ_dP + kk * 8, desc_mnmaj(sK, BN, kk), id_pv, 1);
         }
         mma_commit(&M.empty[st]);
         const uint32_t my = ce[st]++;
-        if (t + 1 < nk && !(ok = issue_s(t + 1))) break;
+        if (t + 1 < nk) issue_dP(t + 1);
         if (t + 2 < nk) {
           if (!(ok = mbar_wait(&M.empty[st], my & 1, abort))) break;
           load_kv(t + 2);
@@ -660,31 +672,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < kCompute) {
       const float Dv = M.Dr[tid];
       for (int t = 0; ok && t < nk; ++t) {
+        const uint32_t sb = (t & 1) ? kQ_S2 : kQ_S;
         if (!(ok = wwait(&M.s_ready, ph_s & 1, abort))) break;
         ++ph_s;
         tc_fence_after();
         const int blk = M.list[t];
         const int kvalid = min(BN, p.N - blk * BN);
-        // dS as bf16 hi (over the read S columns) + lo (over the read dP
-        // columns): dq sums dS K over the kept keys with cancellation, where
+        // phase 1 (while dq += dS(t - 1) K and dP run): P in fp32 over S
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(trow + sb + c * 32, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c0 = c * 32 + e;
+            sv[e] = __float_as_uint(c0 < kvalid ? fast_exp2(__uint_as_float(sv[e]) * p.scale_log2 - lse2) : 0.f);
+          }
+          tmem_st32(trow + sb + c * 32, sv);
+        }
+        tmem_wait_st();
+        if (!(ok = wwait(&M.d_ready, ph_d & 1, abort))) break;
+        ++ph_d;
+        tc_fence_after();
+        // phase 2: dS as bf16 hi (over the read P columns) + lo (over the read
+        // dP columns): dq sums dS K over the kept keys with cancellation, where
         // the bf16 rounding of dS alone is ~2^-9 of sum |dS K|
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t sv[32], dv[32], pk[16], pl[16];
-          tmem_ld32(trow + kQ_S + c * 32, sv);
+          tmem_ld32(trow + sb + c * 32, sv);
           tmem_ld32(trow + kQ_dP + c * 32, dv);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const int c0 = c * 32 + 2 * e;
-            const float p0 = c0 < kvalid ? fast_exp2(__uint_as_float(sv[2 * e]) * p.scale_log2 - lse2) : 0.f;
-            const float p1 = c0 + 1 < kvalid ? fast_exp2(__uint_as_float(sv[2 * e + 1]) * p.scale_log2 - lse2) : 0.f;
+            const float p0 = __uint_as_float(sv[2 * e]), p1 = __uint_as_float(sv[2 * e + 1]);
             const float d0 = p0 * (__uint_as_float(dv[2 * e]) - Dv) * p.scale;
             const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - Dv) * p.scale;
             pk[e] = pack_bf16(d0, d1);
             pl[e] = pack_bf16(d0 - bf16_lo(pk[e]), d1 - bf16_hi(pk[e]));
           }
-          tmem_st16(trow + kQ_S + c * 16, pk);
+          tmem_st16(trow + sb + c * 16, pk);
           tmem_st16(trow + kQ_dP + c * 16, pl);
         }
         tmem_wait_st();
