@@ -787,7 +787,7 @@ struct KLayout {
 };
 
 struct KMisc {
-  uint64_t load, mma, s_ready, p_ready, full[2], empty[2];
+  uint64_t load, mma, s_ready, p_ready, full[2], empty[2], d_ready;
   uint32_t tmem;
   int abort;
   int nkeep;
@@ -828,6 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&M.full[i], 1);
       mbar_init(&M.empty[i], 1);
     }
+    mbar_init(&M.d_ready, 1);
     M.abort = 0;
     fence_barrier_init();
   }
@@ -848,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tm = M.tmem;
   const uint32_t trow = tm + ((uint32_t)((warp & 3) * 32) << 16);
-  uint32_t ph_load = 0, ph_mma = 0, ph_s = 0, ph_p = 0, ph_full[2] = {0, 0}, ce[2] = {0, 0};
+  uint32_t ph_load = 0, ph_mma = 0, ph_s = 0, ph_p = 0, ph_full[2] = {0, 0}, ce[2] = {0, 0}, ph_d = 0;
   float dph[R];
 #pragma unroll
   for (int i = 0; i < R; ++i) dph[i] = 0.f;
@@ -893,22 +894,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                       h, a * BM, b);
         }
       };
-      auto issue_s = [&](int t) -> bool {
+      auto issue_S = [&](int t) -> bool {
         const int st = t & 1;
         if (!mbar_wait(&M.full[st], ph_full[st] & 1, abort)) return false;
         ++ph_full[st];
         tc_fence_after();
-        const uint32_t sQa = smem_u32(smem + L::ring_off + (2 * st) * TILE), sOa = sQa + TILE;
-        for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t sQa = smem_u32(smem + L::ring_off + (2 * st) * TILE);
+        for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tm + kK_S, desc_kmaj(sK, BN, kk), desc_kmaj(sQa, BM, kk), id_dd, kk > 0);
-          mma_ss(tm + kK_dP, desc_kmaj(sV, BN, kk), desc_kmaj(sOa, BM, kk), id_dd, kk > 0);
-        }
         mma_commit(&M.s_ready);
         return true;
       };
+      auto issue_dP = [&](int t) {
+        const uint32_t sOa = smem_u32(smem + L::ring_off + (2 * (t & 1) + 1) * TILE);
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tm + kK_dP, desc_kmaj(sV, BN, kk), desc_kmaj(sOa, BM, kk), id_dd, kk > 0);
+        mma_commit(&M.d_ready);
+      };
       for (int t = 0; t < min(nkeep, 2); ++t) load_q(t);
       ok = mbar_wait(&M.load, ph_load & 1, abort);
-      if (ok && nkeep > 0) ok = issue_s(0);
+      if (ok && nkeep > 0 && (ok = issue_S(0))) issue_dP(0);
+      // per keeper t: dV += P^T dO and dK's lo part (they read the S^T
+      // columns), then S^T(t + 1) over those columns (the next keeper's
+      // exponentials need only it), then dK's hi part (it reads the dP^T
+      // columns), then dP^T(t + 1) over them
       for (int t = 0; ok && t < nkeep; ++t) {
         const int st = t & 1;
         if (!(ok = mbar_wait(&M.p_ready, ph_p & 1, abort))) break;
@@ -917,12 +926,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sQa = smem_u32(smem + L::ring_off + (2 * st) * TILE), sOa = sQa + TILE;
         for (int kk = 0; kk < BM / 16; ++kk) {
           mma_ts(tm + kK_dV, tm + kK_S + kk * 8, desc_mnmaj(sOa, BM, kk), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tm + kK_dK, tm + kK_dP + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tm + kK_dK, tm + kK_S + 64 + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, 1u);
+          mma_ts(tm + kK_dK, tm + kK_S + 64 + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
+        if (t + 1 < nkeep && !(ok = issue_S(t + 1))) break;
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tm + kK_dK, tm + kK_dP + kk * 8, desc_mnmaj(sQa, BM, kk), id_pv, 1u);
         mma_commit(&M.empty[st]);
         const uint32_t my = ce[st]++;
-        if (t + 1 < nkeep && !(ok = issue_s(t + 1))) break;
+        if (t + 1 < nkeep) issue_dP(t + 1);
         if (t + 2 < nkeep) {
           if (!(ok = mbar_wait(&M.empty[st], my & 1, abort))) break;
           load_q(t + 2);
@@ -948,9 +959,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++ph_s;
         if (!ok) continue;
         tc_fence_after();
-        // P^T (bf16) over the read S^T columns [0, 64), dS^T hi over the read
-        // dP^T columns [0, 64), dS^T lo (held until every S^T column is read)
-        // over S^T columns [64, 128)
+        // phase 1 (while dK's hi part and dP^T run): P^T in fp32 over S^T
+#pragma unroll 1
+        for (int c = 0; c < BM / 32; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(trow + kK_S + c * 32, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            sv[e] = __float_as_uint(fast_exp2(__uint_as_float(sv[e]) * p.scale_log2 - M.lse2[st][c * 32 + e]));
+          tmem_st32(trow + kK_S + c * 32, sv);
+        }
+        tmem_wait_st();
+        if (ok) ok = wwait(&M.d_ready, ph_d & 1, abort);
+        ++ph_d;
+        if (!ok) continue;
+        tc_fence_after();
+        // phase 2: P^T (bf16) over the read P^T columns [0, 64), dS^T hi over
+        // the read dP^T columns [0, 64), dS^T lo (held until every P^T column
+        // is read) over columns [64, 128)
         uint32_t dl[64];
 #pragma unroll
         for (int c = 0; c < BM / 32; ++c) {
@@ -961,8 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int q0 = c * 32 + 2 * e;
-            const float p0 = fast_exp2(__uint_as_float(sv[2 * e]) * p.scale_log2 - M.lse2[st][q0]);
-            const float p1 = fast_exp2(__uint_as_float(sv[2 * e + 1]) * p.scale_log2 - M.lse2[st][q0 + 1]);
+            const float p0 = __uint_as_float(sv[2 * e]), p1 = __uint_as_float(sv[2 * e + 1]);
             pp[e] = pack_bf16(p0, p1);
             const float d0 = p0 * (__uint_as_float(dv[2 * e]) - M.Dr[st][q0]) * p.scale;
             const float d1 = p1 * (__uint_as_float(dv[2 * e + 1]) - M.Dr[st][q0 + 1]) * p.scale;
