@@ -488,7 +488,7 @@ def config_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) 
     return rep
 
 
-def backward_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int) -> dict:
+def backward_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int, heads: int = 0) -> dict:
     """Training on one attention workload: the training forward (which also
     saves the output residual, log-sum-exp and linear denominator) and the
     backward (transposed mask, query-major and key-major tcgen05 passes,
@@ -502,6 +502,8 @@ def backward_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int
     from sparse_linear_attention_mean_b200 import binding as rb
     from sparse_linear_attention_mean_b200 import synth
     w = synth.WORKLOADS[wid]
+    if heads:
+        w = synth.custom_workload(w, H=heads)
     shape = rb.Shape.of(w)
     inp = synth.make_inputs(w)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).cuda()
@@ -531,7 +533,7 @@ def backward_report(wid: int, stream, peaks: dict, flush, warmup: int, reps: int
     t_b = [x[0] for x in _timed_reps(f_bwd, stream, flush, warmup, reps)]
     assert int(err.item()) == 0
     flop_fwd = w.sparse_flops()
-    rep = {"workload": w.name, "reps": reps, "warmup": warmup, "l2": "256 MB flush before each rep",
+    rep = {"workload": w.name, "H": w.H, "reps": reps, "warmup": warmup, "l2": "256 MB flush before each rep",
            "train_forward_ms_p50": _pct(t_f, 50), "train_forward_ms_p95": _pct(t_f, 95),
            "backward_ms_p50": _pct(t_b, 50), "backward_ms_p95": _pct(t_b, 95)}
     rep["train_forward_tflops"] = flop_fwd / (rep["train_forward_ms_p50"] * 1e-3) / 1e12
@@ -728,7 +730,7 @@ def main() -> int:
         import torch
         stream = torch.cuda.current_stream()
         print(json.dumps({"training": backward_report(args.workload, stream, measured_peaks(), L2Flush(),
-                                                      args.warmup, args.steps)}))
+                                                      args.warmup, args.steps, args.heads)}))
         return 0
     return run_gpu(args)
 
