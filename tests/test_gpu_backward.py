@@ -124,16 +124,18 @@ def test_backward_dense_limit_every_block_kept():
     assert torch.all(dP == 0) and torch.all(dg == 0)
 
 
-@pytest.mark.parametrize("cfg,heads", [(1, [0, 11]), (2, [39]), (3, [0])])
-def test_backward_workloads(cfg, heads):
+@pytest.mark.parametrize("cfg,heads,gate_scale", [(1, [0, 11], 1.0), (2, [39], 1.0), (3, [0], 1.0), (3, [7], 1000.0)])
+def test_backward_workloads(cfg, heads, gate_scale):
     """Wan2.1-1.3B 480P (all rows of two heads), 14B 480P (all rows of the
-    last head) and 14B 720P (all rows of head 0), at the nominal gate."""
+    last head) and 14B 720P (all rows of head 0) at the nominal gate, and
+    all rows of a 720P head at 1000x the gate, where the linear branch's
+    gradients (state gather, complement, 720P rotary table) carry the result."""
     w = synth.WORKLOADS[cfg]
     inp = synth.make_inputs(w)
     idx_ref, _ = ro.select_all(inp, w.block, w.k_b)
-    r = _run(w, inp, idx_ref=idx_ref)
-    worst = _check_heads(w, inp, r, heads)
-    print(f"workload {cfg}: heads {heads}, worst err/bound {worst:.3f}")
+    r = _run(w, inp, gate_scale, idx_ref=idx_ref)
+    worst = _check_heads(w, inp, r, heads, gate_scale)
+    print(f"workload {cfg}: heads {heads}, gate x{gate_scale:g}, worst err/bound {worst:.3f}")
 
 
 def test_backward_is_deterministic():
